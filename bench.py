@@ -1,0 +1,414 @@
+"""Benchmark of one SVG-EAR attention layer (k-means, permute, probe, route,
+block-sparse attention with compensation) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ear|reference]
+                    [--workload wan|hunyuan|mid|tiny] [--no-cpu-baseline] [--no-e2e]
+
+A step is the whole hot path over one synthetic layer whose inputs are
+already resident in HBM.  The default workload is the Wan2.x-shaped layer
+(40 heads, 75,600 tokens, d = 128, bf16, C_q = 100, C_k = 500, 5 k-means
+iterations, density 0.10).  Inputs (2.3 GB per step) are larger than the
+126 MB L2, so no explicit flush runs between steps.
+
+N > 1 (under torchrun): every rank runs an independent layer (its own seeded
+heads); no collective touches the data path.  Timing is bracketed by a
+barrier and a device synchronize, and the reported time is the max over
+ranks.  `value` = milliseconds per layer for the whole job = max step time /
+layers processed by all ranks per step.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from clustered_block_sparse_b200 import inputs as gen  # noqa: E402
+
+METRIC = "EAR attention ms/layer & tensor-pipe % of peak, Wan-shape 75.6k tok, density 0.10"
+WORKLOADS = {"tiny": gen.TINY, "mid": gen.MID, "wan": gen.WAN, "hunyuan": gen.HUNYUAN}
+STAGES = ("kmeans", "permute", "probe", "route", "attention")
+
+
+# --------------------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ear_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        sm = [r[0] for r in rows]
+        loaded = [r[0] for r in rows if r[2] > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def flops_of(w, exact_pairs_total: int, comp_terms_total: int) -> dict:
+    """Algorithmic work: QK^T and PV (2 flops per MAC each) per exact pair and per
+    compensated (query, centroid) term; k-means and probe distance GEMMs."""
+    d = w.d
+    return {
+        "attention": 4.0 * d * (exact_pairs_total + comp_terms_total),
+        "exact": 4.0 * d * exact_pairs_total,
+        "dense_equiv": 4.0 * d * w.n * w.n * w.heads,
+        "kmeans": 2.0 * w.n * (w.c_q + w.c_k) * d * w.iters * w.heads,
+        "probe": 2.0 * w.c_q * w.n * d * w.heads,
+    }
+
+
+def attention_bytes(w) -> float:
+    """Bytes the attention step must move once: Q, K, V in and O out."""
+    return 4.0 * w.heads * w.n * w.d * (2 if w.dtype == "bf16" else 4)
+
+
+# --------------------------------------------------------------------------- oracle arm
+def oracle_sample(w, layer, query_fraction=0.05, seed=0):
+    """Time the fp64 oracle on head 0: every step in full except attention,
+    which runs on a seeded sample of the queries.  Returns (ms per layer
+    extrapolated, seconds actually spent, description)."""
+    from oracle import ear_oracle as eo
+
+    h = 0
+    q, k, v = layer.q[h], layer.k[h], layer.v[h]
+    s = 1.0 / math.sqrt(w.d)
+    t0 = time.perf_counter()
+    qc, ql, qn = eo.kmeans(q, layer.q_init[h], w.iters)
+    kc, kl, kn = eo.kmeans(k, layer.k_init[h], w.iters)
+    eo.permute(ql, w.c_q)
+    eo.permute(kl, w.c_k)
+    vm = eo.segment_mean(v, kl, w.c_k)
+    e = eo.probe(qc, qn, k, kl, kc, kn, s)
+    exact, _ = eo.route(e, qn, kn, w.n, w.n, w.density)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(seed)
+    nsel = max(1, int(round(query_fraction * w.n)))
+    sel = rng.choice(w.n, nsel, replace=False)
+    eo.attention(q[sel], k, v, ql[sel], kl, kc, vm, kn, exact, s)
+    t2 = time.perf_counter()
+    per_head = (t1 - t0) + (t2 - t1) * (w.n / nsel)
+    desc = (f"head 0 of {w.heads}: k-means/permute/probe/route in full, attention on "
+            f"{nsel} of {w.n} queries; extrapolated x{w.n / nsel:.1f} (attention) and "
+            f"x{w.heads} (heads)")
+    return per_head * w.heads * 1e3, t2 - t0, desc
+
+
+def run_reference(args, w):
+    from oracle import ear_oracle as eo
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    layer = gen.make_layer(w, heads=[0])
+    frac = 0.02 if w.n > 50000 else 1.0
+    for _ in range(args.warmup):
+        oracle_sample(w, layer, frac)
+    vals = []
+    spent = 0.0
+    desc = ""
+    for i in range(args.steps):
+        ms, sec, desc = oracle_sample(w, layer, frac, seed=i)
+        vals.append(ms)
+        spent += sec
+    value = statistics.mean(vals)
+    cores = eo.max_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/layer",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": value,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "ms/layer", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "ms/layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, n_gpus):
+    return {"workload": w.name, "heads": w.heads, "n_q": w.n, "n_k": w.n, "d": w.d,
+            "c_q": w.c_q, "c_k": w.c_k, "kmeans_iters": w.iters, "density": w.density,
+            "ratio_mode": 0, "compensate": True,
+            "l2": "inputs larger than L2 (Q, K, V per step >> 126 MB); no flush",
+            "parallelism": f"{n_gpus} independent replica(s), one layer per rank, no collective"}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_ear(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from clustered_block_sparse_b200 import _native as nat
+    from clustered_block_sparse_b200 import ear
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    distributed = world > 1
+    if distributed:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if distributed:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if not distributed:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    heads = list(range(rank * w.heads, (rank + 1) * w.heads))
+    layer = gen.make_layer(w, heads=heads)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = torch.device("cuda", local)
+    q = torch.from_numpy(layer.q).to(dev, tdt)
+    k = torch.from_numpy(layer.k).to(dev, tdt)
+    v = torch.from_numpy(layer.v).to(dev, tdt)
+    qi = torch.from_numpy(layer.q_init).to(dev)
+    ki = torch.from_numpy(layer.k_init).to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        """One layer; `ev` = 6 events recorded at the stage boundaries."""
+        rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        rec(0)
+        qc, ql, qn = ear.ear_kmeans(q, qi, w.iters)
+        kc, kl, kn = ear.ear_kmeans(k, ki, w.iters)
+        rec(1)
+        qp, qo, qx, _ = ear.ear_permute(ql, w.c_q, q)
+        kp, ko, kx, _ = ear.ear_permute(kl, w.c_k, k)
+        _, _, vx, vm = ear.ear_permute(kl, w.c_k, v, seg_mean=True)
+        rec(2)
+        e = ear.ear_probe(qc, qn, kc, kx, ko)
+        rec(3)
+        exact, bo, bl, pairs = ear.ear_route(e, qn, kn, w.n, w.n, w.density)
+        rec(4)
+        ear.ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, out=out)
+        rec(5)
+        return exact, qo, kn, pairs
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ear.ear_get_device_status() != 0:
+        raise RuntimeError("device status latched an error during warm-up")
+
+    # algorithmic work of this layer (routing is deterministic given the inputs)
+    exact, qo, kn, pairs = step()
+    torch.cuda.synchronize()
+    exact_h = exact.cpu().numpy().astype(np.int64)
+    qsz = np.diff(qo.cpu().numpy().astype(np.int64), axis=1)
+    k_sizes = kn.cpu().numpy()
+    pairs_total = int(pairs.sum().item())
+
+    # timed region: K steps with stage events, clocks sampled meanwhile
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    launches0 = nat.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = nat.launch_count() - launches0
+    total_ms = t_start.elapsed_time(t_end)
+    stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, s in enumerate(STAGES)}
+    ms_step = max_over_ranks(total_ms / args.steps)
+    if ear.ear_get_device_status() != 0:
+        raise RuntimeError("device status latched an error in the timed region")
+
+    # compensated (query, centroid) terms: |a| x (non-empty, non-exact key clusters)
+    comp_terms = 0
+    for h in range(exact_h.shape[0]):
+        nonempty = k_sizes[h] > 0
+        comp = ((exact_h[h] == 0) & nonempty[None, :]).sum(axis=1)
+        comp_terms += int((qsz[h] * comp).sum())
+    fl = flops_of(w, pairs_total, comp_terms)
+    peaks = measured_peaks()
+    attn_s = stage_ms["attention"] * 1e-3
+    achieved = fl["attention"] / attn_s / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+
+    # end to end through the public API: pinned host inputs in, output back out
+    e2e = None
+    if not args.no_e2e:
+        e2e = time_e2e(args, w, layer, ear, dev, tdt, stream)
+        e2e["value"] = max_over_ranks(e2e["value"]) / world
+
+    line = {
+        "metric": METRIC,
+        "value": ms_step / world,
+        "unit": "ms/layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded Gaussian-mixture / smoothed-field tokens; no model weights)",
+        "config": config_of(w, world),
+        "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
+        "overhead_frac": (stage_ms["kmeans"] + stage_ms["probe"] + stage_ms["route"]) /
+                         sum(stage_ms.values()),
+        "tflops": {"attention_algorithmic": achieved,
+                   "exact_blocks": fl["exact"] / attn_s / 1e12,
+                   "dense_equivalent_layer": fl["dense_equiv"] / (ms_step * 1e-3) / 1e12},
+        "tensor_pipe_pct_of_peak": 100.0 * achieved / peak,
+        "roofline": {"bound": "tensor", "kernel": "ear_attention", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
+                     "traffic": None,
+                     "algorithmic_bytes": attention_bytes(w),
+                     "algorithmic_flops": fl["attention"]},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import ear_oracle as eo
+        base = gen.make_layer(w, heads=[0]) if w.heads > 1 else layer
+        ms, spent, desc = oracle_sample(w, base, 0.05 if w.n > 50000 else 1.0)
+        line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": eo.max_threads(),
+                                "kind": "oracle", "sample": desc, "cpu_seconds": spent}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if distributed:
+        dist.destroy_process_group()
+    return 0
+
+
+def time_e2e(args, w, layer, ear, dev, tdt, stream):
+    import torch
+
+    host = {n: torch.from_numpy(getattr(layer, n)).to(tdt).pin_memory() for n in ("q", "k", "v")}
+    host_init = {n: torch.from_numpy(getattr(layer, n)).pin_memory() for n in ("q_init", "k_init")}
+    o_host = torch.empty(host["q"].shape, dtype=tdt).pin_memory()
+    bufs = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
+    ibufs = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host_init.items()}
+
+    def one():
+        for n in host:
+            bufs[n].copy_(host[n], non_blocking=True)
+        for n in host_init:
+            ibufs[n].copy_(host_init[n], non_blocking=True)
+        res = ear.ear_layer(bufs["q"], bufs["k"], bufs["v"], ibufs["q_init"], ibufs["k_init"],
+                            w.iters, w.density)
+        o_host.copy_(res.o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + \
+        sum(t.numel() * t.element_size() for t in host_init.values())
+    d2h = o_host.numel() * o_host.element_size()
+    return {"value": a.elapsed_time(b) / args.steps, "unit": "ms/layer",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ear", "reference"), default="ear")
+    ap.add_argument("--workload", choices=tuple(WORKLOADS), default="wan")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ear(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,134 @@
+// Internal declarations shared by libear's CUDA translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ear.h"
+
+namespace ear {
+
+// ---------------------------------------------------------------- host side
+// Device address of the per-device status word (resolved once per device).
+int* device_status_word();
+// Counts one kernel launch and checks the launch for a configuration error.
+ear_status after_launch();
+
+#define EAR_TRY(expr)                         \
+  do {                                        \
+    ear_status st_ = (expr);                  \
+    if (st_ != EAR_OK) return st_;            \
+  } while (0)
+
+#define EAR_CUDA(expr)                        \
+  do {                                        \
+    if ((expr) != cudaSuccess) return EAR_ERR_CUDA; \
+  } while (0)
+
+// Carves 256-byte aligned sub-buffers out of a caller workspace; with a null
+// base it only measures.
+struct Carver {
+  char* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    size_t off = (used + 255) & ~size_t(255);
+    used = off + count * sizeof(T);
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Work-list geometry shared by the attention launchers.
+constexpr int kAttnTileRows = 64;  // smallest query tile of any attention kernel
+inline int64_t attn_items_per_slice(int64_t n_q, int32_t c_q) {
+  return ceil_div(n_q, kAttnTileRows) + c_q;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns EAR_OK or EAR_ERR_CUDA; arguments were validated by the ABI.
+size_t kmeans_workspace(int64_t bh, int64_t n, int32_t d, int32_t c);
+ear_status kmeans_run(const void* X, ear_dtype dt, int64_t bh, int64_t n, int32_t d, int32_t c,
+                      int32_t iters, const float* init, float* cent, int32_t* labels,
+                      int32_t* counts, void* ws, cudaStream_t s);
+
+size_t permute_workspace(int64_t bh, int64_t n, int32_t c);
+ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, int32_t* perm,
+                       int32_t* offsets, const void* X, void* X_perm, ear_dtype dt, int32_t d,
+                       float* seg_mean, void* ws, cudaStream_t s);
+
+size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
+ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
+                     ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
+                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws, cudaStream_t s);
+
+size_t route_workspace(int64_t bh, int32_t c_q, int32_t c_k);
+ear_status route_run(const float* E, const int32_t* qn, const int32_t* kn, int64_t bh,
+                     int64_t budget, int32_t c_q, int32_t c_k, int32_t mode, uint8_t* exact,
+                     int32_t* blk_off, int32_t* blk_list, int64_t* pairs, void* ws,
+                     cudaStream_t s);
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  ear_dtype dtype;
+  const int32_t* q_off;
+  const int32_t* k_off;
+  const int32_t* q_perm;
+  const float* k_cent;
+  const float* v_cent;
+  const uint8_t* exact;
+  const int32_t* blk_off;
+  const int32_t* blk_list;
+  int64_t bh, n_q, n_k;
+  int32_t d, c_q, c_k;
+  float scale;
+  int32_t flags;
+  void* O;
+  float* lse;
+};
+size_t attention_workspace(int64_t bh, int64_t n_q, int32_t c_q, int32_t c_k);
+ear_status attention_run(const AttnArgs& a, void* ws, cudaStream_t s);
+
+}  // namespace ear
+
+// ---------------------------------------------------------------- device side
+#ifdef __CUDACC__
+namespace ear {
+
+__device__ __forceinline__ void latch(int* status, int code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t u) {
+  return __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+// Round-to-nearest-even fp32 -> bf16 bits (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  uint32_t u = __float_as_uint(f);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+  __device__ __forceinline__ static float load(const float* p, int64_t i) { return p[i]; }
+  __device__ __forceinline__ static void store(float* p, int64_t i, float v) { p[i] = v; }
+};
+template <>
+struct Elem<uint16_t> {
+  __device__ __forceinline__ static float load(const uint16_t* p, int64_t i) {
+    return bf16_to_f32(p[i]);
+  }
+  __device__ __forceinline__ static void store(uint16_t* p, int64_t i, float v) {
+    p[i] = f32_to_bf16(v);
+  }
+};
+
+}  // namespace ear
+#endif

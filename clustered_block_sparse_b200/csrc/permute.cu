@@ -1,0 +1,247 @@
+// Cluster-contiguous permutation (SVG-EAR §3.1: tokens of a cluster are laid
+// out contiguously so the attention map splits into cluster x cluster blocks).
+//
+// A stable counting sort per slice, in 1024-token tiles:
+//  * pm_tile_hist: per (slice, cluster, tile) member counts.
+//  * pm_scan:      one block per slice turns them into the first output
+//                  position of every (cluster, tile) and writes offsets.
+//  * pm_scatter:   each tile walks its 32 warps in order; a warp groups equal
+//                  labels with __match_any_sync, so a token's position is the
+//                  (cluster, tile) cursor plus the number of earlier tokens of
+//                  its cluster - the order within a cluster is token order.
+//  * pm_gather:    X_perm[r] = X[perm[r]], 16-byte vector copies.
+//  * pm_segmean:   per-cluster fp32 mean of the permuted rows (v̄, §4.3), a
+//                  fixed-order reduction.
+#include "ear_internal.cuh"
+
+namespace ear {
+namespace {
+
+constexpr int kTile = 1024;
+
+__global__ void __launch_bounds__(kTile)
+pm_tile_hist(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
+             int32_t* __restrict__ hist, int* status) {
+  const int64_t h = blockIdx.y;
+  const int64_t i = (int64_t)blockIdx.x * kTile + threadIdx.x;
+  if (i >= N) return;
+  int c = labels[h * N + i];
+  if (c < 0 || c >= C) {
+    latch(status, EAR_ERR_DEVICE);
+    return;
+  }
+  atomicAdd(hist + ((h * C + c) * ntiles + blockIdx.x), 1);
+}
+
+__global__ void __launch_bounds__(1024)
+pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int ntiles,
+        int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int64_t h = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  int32_t* hh = hist + h * (int64_t)C * ntiles;
+  int32_t* th = totals + h * (int64_t)C;
+  // per cluster: exclusive prefix over tiles, total in `totals`
+  for (int c = tid; c < C; c += 1024) {
+    int32_t run = 0;
+    for (int t = 0; t < ntiles; ++t) {
+      int32_t v = hh[(int64_t)c * ntiles + t];
+      hh[(int64_t)c * ntiles + t] = run;
+      run += v;
+    }
+    th[c] = run;
+  }
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  // exclusive scan of totals over clusters -> offsets
+  int32_t* oh = offsets + h * (int64_t)(C + 1);
+  for (int base = 0; base < C; base += 1024) {
+    int c = base + tid;
+    int32_t v = c < C ? th[c] : 0;
+    int32_t x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int32_t w = warp_sums[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        int32_t y = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += y;
+      }
+      warp_sums[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    int32_t incl = x + (wid > 0 ? warp_sums[wid - 1] : 0) + carry;
+    if (c < C) oh[c] = incl - v;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+  if (tid == 0) oh[C] = carry;
+  __syncthreads();
+  // cursor of every (cluster, tile) = cluster offset + earlier tiles' members
+  for (int c = tid; c < C; c += 1024) {
+    int32_t o = oh[c];
+    for (int t = 0; t < ntiles; ++t) hh[(int64_t)c * ntiles + t] += o;
+  }
+}
+
+__global__ void __launch_bounds__(kTile)
+pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
+           int32_t* __restrict__ cursor, int32_t* __restrict__ perm) {
+  const int64_t h = blockIdx.y;
+  const int tile = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int64_t i = (int64_t)tile * kTile + tid;
+  int c = -1;
+  if (i < N) {
+    c = labels[h * N + i];
+    if (c < 0 || c >= C) c = -1;
+  }
+  const unsigned group = __match_any_sync(0xffffffffu, c);
+  const int leader = __ffs(group) - 1;
+  const int before = __popc(group & ((1u << lane) - 1u));
+  int32_t* cur = cursor + (h * C + (c < 0 ? 0 : c)) * (int64_t)ntiles + tile;
+  for (int w = 0; w < 32; ++w) {
+    if (wid == w) {
+      int32_t base = 0;
+      if (lane == leader && c >= 0) base = *cur;
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (c >= 0) {
+        perm[h * N + base + before] = (int32_t)i;
+        if (lane == leader) *cur = base + __popc(group);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void pm_gather(const uint4* __restrict__ X, uint4* __restrict__ Xp,
+                          const int32_t* __restrict__ perm, int64_t N, int row_vecs,
+                          int64_t rows_total, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t g = warp; g < rows_total; g += nwarps) {
+    const int64_t h = g / N;
+    const int32_t src = perm[g];
+    if (src < 0 || src >= N) {
+      if (lane == 0) latch(status, EAR_ERR_DEVICE);
+      continue;
+    }
+    const uint4* s = X + (h * N + src) * row_vecs;
+    uint4* dst = Xp + g * row_vecs;
+    for (int v = lane; v < row_vecs; v += 32) dst[v] = s[v];
+  }
+}
+
+// block: 256 threads = (256 / (D/4)) row groups x (D/4) column quads
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+pm_segmean(const T* __restrict__ Xp, const int32_t* __restrict__ offsets, int64_t N, int C,
+           float* __restrict__ mean) {
+  constexpr int kQuads = D / 4;
+  constexpr int kGroups = 256 / kQuads;
+  __shared__ float4 part[kGroups][kQuads];
+  const int64_t h = blockIdx.y;
+  const int c = blockIdx.x;
+  const int q = threadIdx.x % kQuads, g = threadIdx.x / kQuads;
+  const int32_t* oh = offsets + h * (int64_t)(C + 1);
+  const int32_t r0 = oh[c], r1 = oh[c + 1];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const T* xh = Xp + h * N * D;
+  for (int64_t r = r0 + g; r < r1; r += kGroups) {
+    const T* row = xh + r * D + q * 4;
+    acc.x += Elem<T>::load(row, 0);
+    acc.y += Elem<T>::load(row, 1);
+    acc.z += Elem<T>::load(row, 2);
+    acc.w += Elem<T>::load(row, 3);
+  }
+  part[g][q] = acc;
+  __syncthreads();
+  if (g == 0) {
+    float4 s = part[0][q];
+    for (int k = 1; k < kGroups; ++k) {
+      s.x += part[k][q].x;
+      s.y += part[k][q].y;
+      s.z += part[k][q].z;
+      s.w += part[k][q].w;
+    }
+    const int32_t n = r1 - r0;
+    float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n > 0) {
+      const float fn = (float)n;
+      m = make_float4(s.x / fn, s.y / fn, s.z / fn, s.w / fn);
+    }
+    reinterpret_cast<float4*>(mean + (h * C + c) * (int64_t)D)[q] = m;
+  }
+}
+
+struct PmWs {
+  int32_t* hist;
+  int32_t* totals;
+};
+
+PmWs carve(Carver& cv, int64_t bh, int64_t n, int32_t c) {
+  PmWs w;
+  const int64_t ntiles = ceil_div(n, kTile);
+  w.hist = cv.take<int32_t>((size_t)bh * c * ntiles);
+  w.totals = cv.take<int32_t>((size_t)bh * c);
+  return w;
+}
+
+template <typename T, int D>
+ear_status segmean_t(const void* Xp, const int32_t* offsets, int64_t bh, int64_t n, int32_t c,
+                     float* mean, cudaStream_t s) {
+  pm_segmean<T, D><<<dim3((unsigned)c, (unsigned)bh), 256, 0, s>>>((const T*)Xp, offsets, n, c,
+                                                                   mean);
+  return after_launch();
+}
+
+}  // namespace
+
+size_t permute_workspace(int64_t bh, int64_t n, int32_t c) {
+  Carver cv(nullptr);
+  carve(cv, bh, n, c);
+  return cv.used;
+}
+
+ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, int32_t* perm,
+                       int32_t* offsets, const void* X, void* X_perm, ear_dtype dt, int32_t d,
+                       float* seg_mean, void* ws, cudaStream_t s) {
+  Carver cv(ws);
+  PmWs w = carve(cv, bh, n, c);
+  int* status = device_status_word();
+  const int ntiles = (int)ceil_div(n, kTile);
+  const dim3 tgrid((unsigned)ntiles, (unsigned)bh);
+  EAR_CUDA(cudaMemsetAsync(w.hist, 0, sizeof(int32_t) * bh * c * ntiles, s));
+  EAR_CUDA(cudaMemsetAsync(perm, 0xff, sizeof(int32_t) * bh * n, s));
+  pm_tile_hist<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, status);
+  EAR_TRY(after_launch());
+  pm_scan<<<(unsigned)bh, 1024, 0, s>>>(w.hist, w.totals, c, ntiles, offsets);
+  EAR_TRY(after_launch());
+  pm_scatter<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, perm);
+  EAR_TRY(after_launch());
+  if (X == nullptr) return EAR_OK;
+  const int elem = dt == EAR_F32 ? 4 : 2;
+  const int row_vecs = d * elem / 16;
+  const int64_t rows_total = bh * n;
+  const unsigned ggrid = (unsigned)std::min<int64_t>(ceil_div(rows_total, 8), 148 * 64);
+  pm_gather<<<ggrid, 256, 0, s>>>((const uint4*)X, (uint4*)X_perm, perm, n, row_vecs, rows_total,
+                                  status);
+  EAR_TRY(after_launch());
+  if (seg_mean == nullptr) return EAR_OK;
+  if (dt == EAR_F32)
+    return d == 64 ? segmean_t<float, 64>(X_perm, offsets, bh, n, c, seg_mean, s)
+                   : segmean_t<float, 128>(X_perm, offsets, bh, n, c, seg_mean, s);
+  return d == 64 ? segmean_t<uint16_t, 64>(X_perm, offsets, bh, n, c, seg_mean, s)
+                 : segmean_t<uint16_t, 128>(X_perm, offsets, bh, n, c, seg_mean, s);
+}
+
+}  // namespace ear

@@ -1,0 +1,197 @@
+"""Python binding of libear: one function per C entry point, same names.
+
+Argument marshalling only: every step runs in libear's CUDA kernels.  Tensors
+are torch CUDA tensors (torch provides device memory and the stream); outputs
+are allocated here when not passed in.  Errors raise ``EarError``.
+
+Citations "SVG-EAR §x" are to "SVG-EAR: Parameter-Free Linear Compensation for
+Sparse Video Generation via Error-aware Routing" (arXiv 2603.08982).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+from . import _native as N
+from ._native import EarError  # noqa: F401  (re-export)
+
+_DT = {torch.float32: N.EAR_F32, torch.bfloat16: N.EAR_BF16}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; libear takes float32 or bfloat16")
+    return _DT[t.dtype]
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def _workspace(op, bh, n_q, n_k, d, c_q, c_k, device):
+    nbytes = N.workspace_bytes(op, bh, n_q, n_k, d, c_q, c_k)
+    if nbytes == 0:
+        return None, 0
+    return torch.empty(nbytes, dtype=torch.uint8, device=device), nbytes
+
+
+def ear_kmeans(x: torch.Tensor, init: torch.Tensor, iters: int):
+    """Lloyd k-means (SVG-EAR §4.1). x [BH,N,d], init [BH,C,d] float32.
+
+    Returns (centroids [BH,C,d] f32, labels [BH,N] i32, counts [BH,C] i32)."""
+    _need(x, "x")
+    _need(init, "init")
+    bh, n, d = x.shape
+    c = init.shape[1]
+    cent = torch.empty((bh, c, d), dtype=torch.float32, device=x.device)
+    labels = torch.empty((bh, n), dtype=torch.int32, device=x.device)
+    counts = torch.empty((bh, c), dtype=torch.int32, device=x.device)
+    ws, nb = _workspace(N.EAR_OP_KMEANS, bh, n, 0, d, c, 0, x.device)
+    N.check("ear_kmeans", N.lib().ear_kmeans(
+        _p(x), _dtype(x), bh, n, d, c, int(iters), _p(init), _p(cent), _p(labels), _p(counts),
+        _p(ws), nb, _stream(x.device)))
+    return cent, labels, counts
+
+
+def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor] = None,
+                seg_mean: bool = False):
+    """Stable cluster-contiguous permutation (SVG-EAR §3.1).
+
+    Returns (perm [BH,N] i32, offsets [BH,C+1] i32, x_perm or None, mean [BH,C,d] f32 or None)."""
+    _need(labels, "labels")
+    bh, n = labels.shape
+    dev = labels.device
+    perm = torch.empty((bh, n), dtype=torch.int32, device=dev)
+    offsets = torch.empty((bh, n_clusters + 1), dtype=torch.int32, device=dev)
+    x_perm = mean = None
+    d, dt = 0, 0
+    if x is not None:
+        _need(x, "x")
+        d, dt = x.shape[2], _dtype(x)
+        x_perm = torch.empty_like(x)
+        if seg_mean:
+            mean = torch.empty((bh, n_clusters, d), dtype=torch.float32, device=dev)
+    ws, nb = _workspace(N.EAR_OP_PERMUTE, bh, n, 0, d, n_clusters, 0, dev)
+    N.check("ear_permute", N.lib().ear_permute(
+        _p(labels), bh, n, n_clusters, _p(perm), _p(offsets), _p(x), _p(x_perm), dt, d, _p(mean),
+        _p(ws), nb, _stream(dev)))
+    return perm, offsets, x_perm, mean
+
+
+def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Optional[float] = None):
+    """E[a,b] = sum_{j in b} (s q̄_a·k_j - s q̄_a·k̄_b)^2 (SVG-EAR §4.2). Returns E [BH,C_q,C_k] f32."""
+    for t, nm in ((q_centroids, "q_centroids"), (q_counts, "q_counts"), (k_centroids, "k_centroids"),
+                  (k_perm, "k_perm"), (k_offsets, "k_offsets")):
+        _need(t, nm)
+    bh, c_q, d = q_centroids.shape
+    c_k = k_centroids.shape[1]
+    n_k = k_perm.shape[1]
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    e = torch.empty((bh, c_q, c_k), dtype=torch.float32, device=k_perm.device)
+    ws, nb = _workspace(N.EAR_OP_PROBE, bh, 0, n_k, d, c_q, c_k, k_perm.device)
+    N.check("ear_probe", N.lib().ear_probe(
+        _p(q_centroids), _p(q_counts), _p(k_centroids), _p(k_perm), _dtype(k_perm), _p(k_offsets),
+        bh, n_k, d, c_q, c_k, ctypes.c_float(s), _p(e), _p(ws), nb, _stream(k_perm.device)))
+    return e
+
+
+def ear_route(e, q_counts, k_counts, n_q: int, n_k: int, density: float, ratio_mode: int = 0):
+    """Greedy error-to-cost routing under the density budget (SVG-EAR §4.2).
+
+    Returns (exact [BH,C_q,C_k] u8, blk_offsets [BH,C_q+1] i32, blk_list [BH,C_q*C_k] i32,
+    exact_pairs [BH] i64)."""
+    _need(e, "E")
+    bh, c_q, c_k = e.shape
+    dev = e.device
+    exact = torch.empty((bh, c_q, c_k), dtype=torch.uint8, device=dev)
+    blk_off = torch.empty((bh, c_q + 1), dtype=torch.int32, device=dev)
+    blk_list = torch.empty((bh, c_q * c_k), dtype=torch.int32, device=dev)
+    pairs = torch.empty((bh,), dtype=torch.int64, device=dev)
+    ws, nb = _workspace(N.EAR_OP_ROUTE, bh, n_q, n_k, 0, c_q, c_k, dev)
+    N.check("ear_route", N.lib().ear_route(
+        _p(e), _p(q_counts), _p(k_counts), bh, n_q, n_k, c_q, c_k, ctypes.c_double(density),
+        int(ratio_mode), _p(exact), _p(blk_off), _p(blk_list), _p(pairs), _p(ws), nb, _stream(dev)))
+    return exact, blk_off, blk_list, pairs
+
+
+def ear_attention(q_perm_x, k_perm_x, v_perm_x, q_offsets, k_offsets, q_perm, k_centroids,
+                  v_centroids, exact, blk_offsets, blk_list, scale: Optional[float] = None,
+                  compensate: bool = True, want_lse: bool = False, out: Optional[torch.Tensor] = None):
+    """Block-sparse attention with linear compensation (SVG-EAR §4.1, §4.3).
+
+    Returns (O [BH,N_q,d] in original query order, lse [BH,N_q] f32 or None)."""
+    bh, n_q, d = q_perm_x.shape
+    n_k = k_perm_x.shape[1]
+    c_q = q_offsets.shape[1] - 1
+    c_k = k_offsets.shape[1] - 1
+    dev = q_perm_x.device
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q_perm_x) if out is None else out
+    lse = torch.empty((bh, n_q), dtype=torch.float32, device=dev) if want_lse else None
+    ws, nb = _workspace(N.EAR_OP_ATTENTION, bh, n_q, n_k, d, c_q, c_k, dev)
+    N.check("ear_attention", N.lib().ear_attention(
+        _p(q_perm_x), _p(k_perm_x), _p(v_perm_x), _dtype(q_perm_x), _p(q_offsets), _p(k_offsets),
+        _p(q_perm), _p(k_centroids), _p(v_centroids), _p(exact), _p(blk_offsets), _p(blk_list),
+        bh, n_q, n_k, d, c_q, c_k, ctypes.c_float(s), N.EAR_COMPENSATE if compensate else 0,
+        _p(o), _p(lse), _p(ws), nb, _stream(dev)))
+    return o, lse
+
+
+def ear_get_device_status(device=None) -> int:
+    """Synchronize the current stream and return (and clear) the latched device status."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    out = ctypes.c_int32(0)
+    N.check("ear_get_device_status", N.lib().ear_get_device_status(ctypes.byref(out), _stream(dev)))
+    return int(out.value)
+
+
+@dataclasses.dataclass
+class LayerResult:
+    o: torch.Tensor
+    lse: Optional[torch.Tensor]
+    q_centroids: torch.Tensor
+    q_labels: torch.Tensor
+    q_counts: torch.Tensor
+    k_centroids: torch.Tensor
+    k_labels: torch.Tensor
+    k_counts: torch.Tensor
+    q_perm: torch.Tensor
+    q_offsets: torch.Tensor
+    k_perm: torch.Tensor
+    k_offsets: torch.Tensor
+    v_mean: torch.Tensor
+    e: torch.Tensor
+    exact: torch.Tensor
+    blk_offsets: torch.Tensor
+    blk_list: torch.Tensor
+    exact_pairs: torch.Tensor
+
+
+def ear_layer(q, k, v, q_init, k_init, iters: int, density: float, ratio_mode: int = 0,
+              compensate: bool = True, want_lse: bool = False, scale: Optional[float] = None,
+              out: Optional[torch.Tensor] = None) -> LayerResult:
+    """One SVG-EAR attention layer: the five entry points in order (SVG-EAR §3.1, §4)."""
+    n_q, n_k = q.shape[1], k.shape[1]
+    qc, ql, qn = ear_kmeans(q, q_init, iters)
+    kc, kl, kn = ear_kmeans(k, k_init, iters)
+    qp, qo, qx, _ = ear_permute(ql, q_init.shape[1], q)
+    kp, ko, kx, _ = ear_permute(kl, k_init.shape[1], k)
+    _, _, vx, vm = ear_permute(kl, k_init.shape[1], v, seg_mean=True)
+    e = ear_probe(qc, qn, kc, kx, ko, scale)
+    exact, bo, bl, pairs = ear_route(e, qn, kn, n_q, n_k, density, ratio_mode)
+    o, lse = ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, scale, compensate,
+                           want_lse, out)
+    return LayerResult(o, lse, qc, ql, qn, kc, kl, kn, qp, qo, kp, ko, vm, e, exact, bo, bl, pairs)

@@ -1,0 +1,219 @@
+/*
+ * ear.h - C ABI of libear, the B200 (sm_100a) SVG-EAR attention hot path.
+ *
+ * The method is SVG-EAR ("SVG-EAR: Parameter-Free Linear Compensation for
+ * Sparse Video Generation via Error-aware Routing", arXiv 2603.08982); the
+ * section cited beside each entry point defines what it computes.
+ *
+ * One attention layer runs five calls, in this order, for all (batch, head)
+ * slices at once ("BH" slices):
+ *   ear_kmeans(Q), ear_kmeans(K)       cluster queries and keys
+ *   ear_permute(Q), (K), (V with K's   make each cluster contiguous
+ *     labels, also producing v̄)
+ *   ear_probe                          per-block compensation-error estimate
+ *   ear_route                          greedy error-to-cost block selection
+ *   ear_attention                      block-sparse exact attention plus
+ *                                      centroid compensation, one softmax
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every array pointer is a DEVICE pointer owned by the caller, contiguous,
+ *    16-byte aligned, row-major.  The library keeps no pointer after a call
+ *    returns and allocates no device or host memory.
+ *  - Token matrices are [BH][N][d]; d is 64 or 128.  Element type is given by
+ *    an ear_dtype: EAR_F32 (float) or EAR_BF16 (bfloat16 bits, uint16).
+ *  - Scratch memory is passed as (ws, ws_bytes); its required size comes from
+ *    ear_workspace_bytes().  Contents need not be initialised and are
+ *    clobbered.  Two calls that run concurrently need separate workspaces.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *    void*; NULL = the legacy default stream).  Outputs are valid once the
+ *    stream reaches the call.
+ *  - Host-side validation runs first.  On any error other than EAR_OK the
+ *    call launches nothing and writes no output.  EAR_ERR_CUDA means a CUDA
+ *    runtime call failed; work enqueued before it by the same call may have
+ *    run.
+ *  - Device-side faults that validation cannot see (a label out of range, an
+ *    offset table that is not monotone, a bounded wait that ran out) do not
+ *    trap: the kernel skips the bad item and latches an error code in a
+ *    per-device status word, read and cleared by ear_get_device_status().
+ *  - N < 2^31 and every cluster count C <= 65536.
+ *  - The library is thread-compatible: calls on different streams may run
+ *    from different host threads.
+ */
+#ifndef EAR_H_
+#define EAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EAR_API __attribute__((visibility("default")))
+#else
+#define EAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  EAR_OK = 0,
+  EAR_ERR_ARG = 1,          /* null pointer, bad size or value; nothing launched     */
+  EAR_ERR_UNSUPPORTED = 2,  /* well-formed but outside what is built (d, dtype, C)   */
+  EAR_ERR_WORKSPACE = 3,    /* ws_bytes smaller than ear_workspace_bytes() says      */
+  EAR_ERR_CUDA = 4,         /* a CUDA runtime call failed                            */
+  EAR_ERR_TIMEOUT = 5,      /* device status: a bounded device-side wait ran out     */
+  EAR_ERR_DEVICE = 6        /* device status: an input index/offset was out of range */
+} ear_status;
+
+typedef enum { EAR_F32 = 0, EAR_BF16 = 1 } ear_dtype;
+
+typedef enum {
+  EAR_OP_KMEANS = 0,
+  EAR_OP_PERMUTE = 1,
+  EAR_OP_PROBE = 2,
+  EAR_OP_ROUTE = 3,
+  EAR_OP_ATTENTION = 4
+} ear_op;
+
+/* ear_attention flags */
+#define EAR_COMPENSATE 1 /* fold skipped blocks in through their centroids (SVG-EAR §4.3);
+                            without it skipped blocks are dropped (the §3.1 baseline)    */
+
+/* Static string naming a status code. */
+EAR_API const char* ear_status_string(ear_status s);
+
+/*
+ * Scratch bytes an entry point needs for the given sizes.
+ *   op = EAR_OP_KMEANS:  rows N = n_q, clusters C = c_q   (n_k, c_k ignored)
+ *   op = EAR_OP_PERMUTE: rows N = n_q, clusters C = c_q   (n_k, c_k ignored)
+ *   op = EAR_OP_PROBE / ROUTE / ATTENTION: all sizes as in those calls.
+ * Returns EAR_ERR_ARG for negative sizes or a null `bytes`.
+ */
+EAR_API ear_status ear_workspace_bytes(ear_op op, int64_t bh, int64_t n_q, int64_t n_k, int32_t d,
+                               int32_t c_q, int32_t c_k, size_t* bytes);
+
+/*
+ * Lloyd k-means of every slice's N rows into C clusters (SVG-EAR §4.1: Q and K
+ * are clustered with "flash k-means"; q̄_i / k̄_j is the mean token of the
+ * cluster holding i / j).
+ *   X          [BH][N][d] dtype       rows to cluster
+ *   init       [BH][C][d] float       initial centroids (e.g. C seeded rows of X)
+ *   centroids  [BH][C][d] float  out  means of the final members; an empty
+ *                                     cluster keeps its previous centroid
+ *   labels     [BH][N] int32     out  cluster of each row from the LAST assignment
+ *   counts     [BH][C] int32     out  members per cluster under `labels`
+ * Each of `iters` (>= 1) iterations assigns every row to the nearest centroid
+ * (squared Euclidean distance; ties go to the lowest index) and then moves
+ * every centroid to the mean of its members.  Assignments are exact: a row
+ * whose fast distance gap is within its rounding bound is re-decided in fp64.
+ * Requires 1 <= C <= min(N, 65536).
+ */
+EAR_API ear_status ear_kmeans(const void* X, ear_dtype dtype, int64_t bh, int64_t n, int32_t d,
+                      int32_t c, int32_t iters, const float* init, float* centroids,
+                      int32_t* labels, int32_t* counts, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Cluster-contiguous permutation (SVG-EAR §3.1: tokens are permuted so that
+ * each cluster is contiguous and the attention map splits into blocks).
+ *   labels   [BH][N] int32        cluster of each token, in [0, C)
+ *   perm     [BH][N] int32   out  perm[r] = original index of permuted row r;
+ *                                 a stable sort by label (ties by index)
+ *   offsets  [BH][C+1] int32 out  first permuted row of each cluster; offsets[C] = N
+ *   X        [BH][N][d] dtype     optional (NULL: only perm/offsets are produced)
+ *   X_perm   [BH][N][d] dtype out X_perm[r] = X[perm[r]]            (needs X)
+ *   seg_mean [BH][C][d] float out optional per-cluster mean of X's rows
+ *                                 (SVG-EAR §4.3: v̄ = mean of V over a key
+ *                                 cluster); zero rows for empty clusters (needs X)
+ * A label outside [0, C) latches EAR_ERR_DEVICE and that token is dropped.
+ */
+EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int32_t c,
+                       int32_t* perm, int32_t* offsets, const void* X, void* X_perm,
+                       ear_dtype dtype, int32_t d, float* seg_mean, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Compensation-error probe (SVG-EAR §4.2 "Error estimation"; §1: query
+ * centroids stand in for individual queries, O(C_q N_k d) work).
+ *   q_centroids [BH][C_q][d] float     q̄_a
+ *   q_counts    [BH][C_q] int32        |a|; rows with |a| = 0 get E = 0
+ *   k_centroids [BH][C_k][d] float     k̄_b
+ *   K_perm      [BH][N_k][d] dtype     keys in cluster-contiguous order
+ *   k_offsets   [BH][C_k+1] int32      cluster b = rows [k_offsets[b], k_offsets[b+1])
+ *   E           [BH][C_q][C_k] float out
+ *       E[a][b] = sum_{j in b} (scale q̄_a·k_j - scale q̄_a·k̄_b)^2
+ *   scale is 1/sqrt(d) for the paper's logits.  Empty key clusters get 0.
+ */
+EAR_API ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
+                     const float* k_centroids, const void* K_perm, ear_dtype dtype,
+                     const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
+                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * Greedy error-to-cost routing under a density budget (SVG-EAR §4.2 "Error
+ * estimation": blocks with the highest error-to-size ratio are computed
+ * exactly until the budget is spent; §4.1: nnz(M) <= rho N_q N_k).
+ *   E          [BH][C_q][C_k] float    probe output
+ *   q_counts   [BH][C_q] int32, k_counts [BH][C_k] int32   cluster sizes
+ *   density    rho in [0, 1]; budget B = floor(rho * (N_q*N_k)) pairs per slice
+ *   ratio_mode 0: E[a][b] / |b|  (the pages' ratio: the block sum of the
+ *                 per-entry estimates, |a| E[a][b], over |a||b|)
+ *              1: E[a][b] / (|a| |b|)
+ *   exact       [BH][C_q][C_k] uint8 out  1 = computed exactly
+ *   blk_offsets [BH][C_q+1] int32    out  CSR row starts into blk_list (per slice)
+ *   blk_list    [BH][C_q*C_k] int32  out  exact key clusters of each query
+ *                                         cluster, ascending
+ *   exact_pairs [BH] int64           out  (query, key) pairs computed exactly
+ * Order: ratio descending (computed in fp64), ties to the lower a*C_k+b.
+ * Blocks with |a||b| = 0 are never exact.  The walk adds |a||b| while the
+ * total stays <= B and stops at the first block that does not fit.
+ */
+EAR_API ear_status ear_route(const float* E, const int32_t* q_counts, const int32_t* k_counts,
+                     int64_t bh, int64_t n_q, int64_t n_k, int32_t c_q, int32_t c_k,
+                     double density, int32_t ratio_mode, uint8_t* exact,
+                     int32_t* blk_offsets, int32_t* blk_list, int64_t* exact_pairs,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse attention with linear compensation (SVG-EAR §4.1 routing mask,
+ * §4.3 Linear Compensation).  For query i of cluster a one softmax runs over
+ *   - exact logits scale q_i·k_j, value v_j, for every key j of every key
+ *     cluster b listed in blk_list for a, and
+ *   - (with EAR_COMPENSATE) for every other non-empty key cluster b, the
+ *     logit scale q_i·k̄_b with weight |b| and value v̄_b.
+ *   Q_perm, K_perm, V_perm [BH][N][d] dtype   cluster-contiguous rows
+ *   q_offsets [BH][C_q+1], k_offsets [BH][C_k+1] int32
+ *   q_perm    [BH][N_q] int32        original index of each permuted query
+ *   k_centroids, v_centroids [BH][C_k][d] float   k̄_b, v̄_b
+ *   exact     [BH][C_q][C_k] uint8, blk_offsets, blk_list   from ear_route
+ *   O   [BH][N_q][d] dtype out  written at ORIGINAL query order
+ *   lse [BH][N_q] float    out  optional natural-log normalizer per query
+ * fp32 inputs are computed in fp32; bf16 inputs on the tensor cores with fp32
+ * accumulation.  A query with no term at all gets O = 0 and lse = -inf.
+ */
+EAR_API ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_perm,
+                         ear_dtype dtype, const int32_t* q_offsets, const int32_t* k_offsets,
+                         const int32_t* q_perm, const float* k_centroids,
+                         const float* v_centroids, const uint8_t* exact,
+                         const int32_t* blk_offsets, const int32_t* blk_list, int64_t bh,
+                         int64_t n_q, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k,
+                         float scale, int32_t flags, void* O, float* lse, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/*
+ * Synchronizes `stream`, then returns in *out the first device-side error
+ * code latched on the current device since the last call (EAR_OK if none)
+ * and clears it.
+ */
+EAR_API ear_status ear_get_device_status(int32_t* out, void* stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+EAR_API uint64_t ear_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EAR_H_ */

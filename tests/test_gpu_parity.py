@@ -1,0 +1,369 @@
+"""GPU parity: every libear entry point against the fp64 CPU oracle on the
+same seeded inputs, step by step (each step given the oracle's inputs to it),
+end to end, on edge cases, and on sampled outputs at the Wan2.x layer size.
+
+Tolerances (tests/parity_util.py): labels, permutations and routed blocks
+bit-exact (a differing label/block only at a 1e-6 relative tie); attention
+max-abs 2e-2 and rel-L2 5e-3 for bf16 inputs, max-abs 1e-4 for fp32.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import parity_util as pu
+from clustered_block_sparse_b200 import ear
+from clustered_block_sparse_b200 import inputs as gen
+from oracle import ear_oracle as eo
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from clustered_block_sparse_b200 import build
+    build.build()
+    yield
+    assert ear.ear_get_device_status() == 0
+
+
+def _tdt(w):
+    return pu.torch_dtype(w.dtype)
+
+
+MID2 = gen.MID.with_(heads=2)
+CONFIGS = {"tiny": gen.TINY, "mid": MID2}
+
+
+@pytest.fixture(scope="module")
+def layers():
+    return {k: gen.make_layer(w) for k, w in CONFIGS.items()}
+
+
+@pytest.fixture(scope="module")
+def oracle_runs(layers):
+    out = {}
+    for k, w in CONFIGS.items():
+        L = layers[k]
+        out[k] = [eo.pipeline(L.q[h], L.k[h], L.v[h], L.q_init[h], L.k_init[h], w.iters, w.density)
+                  for h in range(len(L.heads))]
+    return out
+
+
+# --------------------------------------------------------------------------- k-means
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_kmeans_one_iteration_is_exact_argmin(layers, cfg, which):
+    L = layers[cfg]
+    x = getattr(L, which)
+    init = L.q_init if which == "q" else L.k_init
+    cent, lab, cnt = ear.ear_kmeans(pu.dev(x, _tdt(L.workload)), pu.dev(init), 1)
+    cent, lab, cnt = pu.host(cent), pu.host(lab), pu.host(cnt)
+    for h in range(x.shape[0]):
+        c_ref, l_ref, n_ref = eo.kmeans(x[h], init[h], 1)
+        nbad = pu.assert_labels_exact_or_tie(x[h], init[h], lab[h], l_ref)
+        if nbad == 0:
+            np.testing.assert_array_equal(cnt[h], n_ref)
+            np.testing.assert_allclose(cent[h], c_ref, rtol=0, atol=1e-5 * np.abs(c_ref).max())
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_kmeans_all_iterations(layers, cfg):
+    L = layers[cfg]
+    w = L.workload
+    cent, lab, cnt = ear.ear_kmeans(pu.dev(L.k, _tdt(w)), pu.dev(L.k_init), w.iters)
+    cent, lab, cnt = pu.host(cent), pu.host(lab), pu.host(cnt)
+    for h in range(L.k.shape[0]):
+        c_ref, l_ref, n_ref = eo.kmeans(L.k[h], L.k_init[h], w.iters)
+        c_prev, _, _ = eo.kmeans(L.k[h], L.k_init[h], w.iters - 1)
+        bad = np.nonzero(lab[h] != l_ref)[0]
+        # fp32 centroid sums drift ~1e-7 from the fp64 means; a differing final
+        # label must be a near-tie under the oracle's previous centroids
+        for i in bad:
+            x = L.k[h][i].astype(np.float64)
+            dg = ((x - c_prev[lab[h][i]]) ** 2).sum()
+            dr = ((x - c_prev[l_ref[i]]) ** 2).sum()
+            assert abs(dg - dr) <= 1e-4 * ((x ** 2).sum() + (c_prev[l_ref[i]] ** 2).sum())
+        assert len(bad) <= 1e-3 * L.k.shape[1]
+        assert cnt[h].sum() == L.k.shape[1]
+        if len(bad) == 0:
+            np.testing.assert_array_equal(cnt[h], n_ref)
+            np.testing.assert_allclose(cent[h], c_ref, rtol=0, atol=1e-5 * np.abs(c_ref).max())
+
+
+# --------------------------------------------------------------------------- permutation
+@pytest.mark.parametrize("n,c,dtype,d", [(8192, 128, "bf16", 128), (1000, 7, "f32", 64),
+                                         (3001, 40, "bf16", 64), (5, 3, "f32", 128)])
+def test_permute_matches_oracle(n, c, dtype, d):
+    rng = np.random.default_rng(n + c)
+    bh = 3
+    labels = rng.integers(0, c, (bh, n)).astype(np.int32)
+    labels[labels == c // 2] = 0  # one empty cluster per slice
+    x = gen.round_to_dtype(rng.standard_normal((bh, n, d)), dtype)
+    perm, off, xp, mean = ear.ear_permute(pu.dev(labels), c, pu.dev(x, pu.torch_dtype(dtype)),
+                                          seg_mean=True)
+    perm, off, xp, mean = pu.host(perm), pu.host(off), pu.host(xp), pu.host(mean)
+    for h in range(bh):
+        p_ref, o_ref = eo.permute(labels[h], c)
+        np.testing.assert_array_equal(perm[h], p_ref)
+        np.testing.assert_array_equal(off[h], o_ref)
+        np.testing.assert_array_equal(xp[h], x[h][p_ref])
+        m_ref = eo.segment_mean(x[h], labels[h], c)
+        np.testing.assert_allclose(mean[h], m_ref, rtol=0, atol=1e-6 * max(np.abs(m_ref).max(), 1))
+
+
+def test_permute_bad_label_latches_device_status():
+    labels = np.zeros((1, 100), np.int32)
+    labels[0, 17] = 9  # out of range for C = 4
+    perm, off, _, _ = ear.ear_permute(pu.dev(labels), 4)
+    assert ear.ear_get_device_status() == 6  # EAR_ERR_DEVICE
+    assert ear.ear_get_device_status() == 0  # cleared by the read
+    assert pu.host(off)[0, -1] == 99
+
+
+# --------------------------------------------------------------------------- probe
+def _stack(runs, attr, dtype=None):
+    a = np.stack([getattr(r, attr) for r in runs])
+    return a.astype(dtype) if dtype is not None else a
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_probe_matches_oracle(layers, oracle_runs, cfg):
+    L, runs = layers[cfg], oracle_runs[cfg]
+    w = L.workload
+    s = pu.scale_of(w.d)
+    qc = _stack(runs, "q_cent", np.float32)
+    kc = _stack(runs, "k_cent", np.float32)
+    kx = np.stack([L.k[h][runs[h].k_perm] for h in range(len(runs))])
+    e = ear.ear_probe(pu.dev(qc), pu.dev(_stack(runs, "q_counts", np.int32)), pu.dev(kc),
+                      pu.dev(kx, _tdt(w)), pu.dev(_stack(runs, "k_offsets", np.int32)), s)
+    e = pu.host(e)
+    for h, r in enumerate(runs):
+        e_ref = eo.probe(qc[h], r.q_counts, L.k[h], r.k_labels, kc[h], r.k_counts, s)
+        np.testing.assert_allclose(e[h], e_ref, rtol=2e-5, atol=1e-7 * e_ref.max())
+
+
+# --------------------------------------------------------------------------- route
+def _route_case(e, qn, kn, nq, nk, density, mode):
+    exact, bo, bl, pairs = ear.ear_route(pu.dev(e), pu.dev(qn), pu.dev(kn), nq, nk, density, mode)
+    exact, bo, bl, pairs = pu.host(exact), pu.host(bo), pu.host(bl), pu.host(pairs)
+    for h in range(e.shape[0]):
+        ex_ref, p_ref = eo.route(e[h].astype(np.float64), qn[h], kn[h], nq, nk, density, mode)
+        np.testing.assert_array_equal(exact[h], ex_ref)
+        assert pairs[h] == p_ref
+        o_ref, l_ref = eo.block_lists(ex_ref)
+        np.testing.assert_array_equal(bo[h], o_ref)
+        np.testing.assert_array_equal(bl[h][:o_ref[-1]], l_ref)
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("density", [0.0, 0.05, 0.15, 0.25, 0.6, 1.0])
+def test_route_given_same_error_is_bit_exact(oracle_runs, layers, cfg, mode, density):
+    runs = oracle_runs[cfg]
+    L = layers[cfg]
+    e = _stack(runs, "e", np.float32)
+    _route_case(e, _stack(runs, "q_counts", np.int32), _stack(runs, "k_counts", np.int32),
+                L.q.shape[1], L.k.shape[1], density, mode)
+
+
+@pytest.mark.parametrize("seed", range(3))
+@pytest.mark.parametrize("density", [0.0, 0.01, 0.3, 0.97, 1.0])
+def test_route_ties_and_empty_clusters(seed, density):
+    rng = np.random.default_rng(seed)
+    bh, cq, ck = 4, 37, 300
+    qn = rng.integers(0, 50, (bh, cq)).astype(np.int32)
+    kn = rng.integers(0, 30, (bh, ck)).astype(np.int32)
+    qn[:, 3] = 0
+    kn[:, 7] = 0
+    # few distinct values -> many exact ratio ties, broken by block index
+    e = rng.integers(0, 5, (bh, cq, ck)).astype(np.float32) * np.float32(0.25)
+    e[:, :, 11] = e[:, :, 12]
+    e = e * kn[:, None, :]  # equal E/|b| across many blocks in mode 0
+    e *= (qn[:, :, None] > 0) * (kn[:, None, :] > 0)
+    nq, nk = int(qn.sum(1).max()), int(kn.sum(1).max())
+    for mode in (0, 1):
+        _route_case(e.astype(np.float32), qn, kn, nq, nk, density, mode)
+
+
+# --------------------------------------------------------------------------- attention
+def _attention_inputs(L, runs):
+    q = np.stack([L.q[h][r.q_perm] for h, r in enumerate(runs)])
+    k = np.stack([L.k[h][r.k_perm] for h, r in enumerate(runs)])
+    v = np.stack([L.v[h][r.k_perm] for h, r in enumerate(runs)])
+    return q, k, v
+
+
+def _run_attention(L, runs, compensate, exact=None, lists=None):
+    w = L.workload
+    t = _tdt(w)
+    q, k, v = _attention_inputs(L, runs)
+    ex = _stack(runs, "exact") if exact is None else exact
+    if lists is None:
+        bo = _stack(runs, "blk_offsets", np.int32)
+        bl = np.stack([np.pad(r.blk_list, (0, ex.shape[1] * ex.shape[2] - len(r.blk_list)))
+                       for r in runs]).astype(np.int32)
+    else:
+        bo, bl = lists
+    o, lse = ear.ear_attention(
+        pu.dev(q, t), pu.dev(k, t), pu.dev(v, t), pu.dev(_stack(runs, "q_offsets", np.int32)),
+        pu.dev(_stack(runs, "k_offsets", np.int32)), pu.dev(_stack(runs, "q_perm", np.int32)),
+        pu.dev(_stack(runs, "k_cent", np.float32)), pu.dev(_stack(runs, "v_mean", np.float32)),
+        pu.dev(np.ascontiguousarray(ex)), pu.dev(bo), pu.dev(bl), pu.scale_of(w.d), compensate,
+        want_lse=True)
+    return pu.host(o), pu.host(lse)
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+@pytest.mark.parametrize("compensate", [True, False])
+def test_attention_given_same_mask(layers, oracle_runs, cfg, compensate):
+    L, runs = layers[cfg], oracle_runs[cfg]
+    w = L.workload
+    o, lse = _run_attention(L, runs, compensate)
+    for h, r in enumerate(runs):
+        o_ref, lse_ref = eo.attention(L.q[h], L.k[h], L.v[h], r.q_labels, r.k_labels, r.k_cent,
+                                      r.v_mean, r.k_counts, r.exact, pu.scale_of(w.d), compensate)
+        ok = np.isfinite(lse_ref)
+        pu.assert_attention_close(o[h][ok], o_ref[ok], w.dtype)
+        assert np.all(o[h][~ok] == 0) and np.all(np.isneginf(lse[h][~ok]))
+        np.testing.assert_allclose(lse[h][ok], lse_ref[ok], rtol=0, atol=2e-3 if w.dtype == "bf16" else 1e-5)
+
+
+# --------------------------------------------------------------------------- whole layer
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_layer_end_to_end(layers, oracle_runs, cfg):
+    L, runs = layers[cfg], oracle_runs[cfg]
+    w = L.workload
+    t = _tdt(w)
+    res = ear.ear_layer(pu.dev(L.q, t), pu.dev(L.k, t), pu.dev(L.v, t), pu.dev(L.q_init),
+                        pu.dev(L.k_init), w.iters, w.density, want_lse=True)
+    o = pu.host(res.o)
+    qlab, klab = pu.host(res.q_labels), pu.host(res.k_labels)
+    exact, e = pu.host(res.exact), pu.host(res.e)
+    pairs = pu.host(res.exact_pairs)
+    budget = math.floor(w.density * float(L.q.shape[1] * L.k.shape[1]))
+    for h, r in enumerate(runs):
+        assert pairs[h] <= budget
+        assert (qlab[h] != r.q_labels).mean() <= 1e-3 and (klab[h] != r.k_labels).mean() <= 1e-3
+        # blocks may differ only at ratio ties (the centroids carry fp32 rounding)
+        diff = np.argwhere(exact[h] != r.exact)
+        if len(diff):
+            rr = pu.route_ratio(r.e, r.q_counts, r.k_counts, 0)
+            cut = rr[r.exact.astype(bool)].min()
+            for a, b in diff:
+                assert abs(rr[a, b] - cut) <= 1e-4 * cut
+        same_rows = (exact[h] == r.exact).all(axis=1)
+        keep = (qlab[h] == r.q_labels) & same_rows[r.q_labels]
+        assert keep.mean() > 0.9
+        pu.assert_attention_close(o[h][keep], r.o[keep], w.dtype)
+        # E against the oracle's probe with the GPU's own centroids and labels
+        qc, kc = pu.host(res.q_centroids)[h], pu.host(res.k_centroids)[h]
+        e_ref = eo.probe(qc, pu.host(res.q_counts)[h], L.k[h], klab[h], kc,
+                         pu.host(res.k_counts)[h], pu.scale_of(w.d))
+        np.testing.assert_allclose(e[h], e_ref, rtol=2e-5, atol=1e-7 * e_ref.max())
+
+
+# --------------------------------------------------------------------------- edge cases
+def _dense(q, k, v, s):
+    z = s * q.astype(np.float64) @ k.astype(np.float64).T
+    z -= z.max(1, keepdims=True)
+    p = np.exp(z)
+    return (p / p.sum(1, keepdims=True)) @ v.astype(np.float64)
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128), ("bf16", 64), ("f32", 128)])
+def test_full_density_ragged_unequal_lengths_is_dense(dtype, d):
+    rng = np.random.default_rng(5)
+    nq, nk, cq, ck = 701, 1000, 9, 23
+    q = gen.round_to_dtype(rng.standard_normal((2, nq, d)), dtype)
+    k = gen.round_to_dtype(rng.standard_normal((2, nk, d)), dtype)
+    v = gen.round_to_dtype(rng.standard_normal((2, nk, d)), dtype)
+    qi = np.ascontiguousarray(q[:, :cq])
+    ki = np.ascontiguousarray(k[:, :ck])
+    t = pu.torch_dtype(dtype)
+    res = ear.ear_layer(pu.dev(q, t), pu.dev(k, t), pu.dev(v, t), pu.dev(qi), pu.dev(ki), 3, 1.0)
+    assert (pu.host(res.exact_pairs) == nq * nk).all()
+    o = pu.host(res.o)
+    for h in range(2):
+        pu.assert_attention_close(o[h], _dense(q[h], k[h], v[h], 1 / math.sqrt(d)), dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_zero_density_one_key_cluster_is_mean_value(dtype):
+    rng = np.random.default_rng(6)
+    q = gen.round_to_dtype(rng.standard_normal((1, 300, 128)), dtype)
+    k = gen.round_to_dtype(rng.standard_normal((1, 257, 128)), dtype)
+    v = gen.round_to_dtype(rng.standard_normal((1, 257, 128)), dtype)
+    t = pu.torch_dtype(dtype)
+    res = ear.ear_layer(pu.dev(q, t), pu.dev(k, t), pu.dev(v, t), pu.dev(q[:, :4].copy()),
+                        pu.dev(k[:, :1].copy()), 2, 0.0)
+    assert pu.host(res.exact).sum() == 0
+    mean = v[0].astype(np.float64).mean(0)
+    tol = 1e-4 if dtype == "f32" else 1e-2
+    np.testing.assert_allclose(pu.host(res.o)[0], np.broadcast_to(mean, (300, 128)), atol=tol)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("density", [0.0, 0.2])
+def test_singleton_key_clusters_and_empty_clusters(dtype, density):
+    """C_k = N_k with init = the keys (compensation exact) plus duplicated init
+    rows on the query side (clusters that stay empty)."""
+    rng = np.random.default_rng(8)
+    nq, nk, d = 200, 256, 64
+    q = gen.round_to_dtype(rng.standard_normal((1, nq, d)), dtype)
+    k = gen.round_to_dtype(rng.standard_normal((1, nk, d)), dtype)
+    v = gen.round_to_dtype(rng.standard_normal((1, nk, d)), dtype)
+    qi = np.concatenate([q[:, :5], q[:, :5]], axis=1)  # clusters 5..9 duplicate 0..4: empty
+    t = pu.torch_dtype(dtype)
+    res = ear.ear_layer(pu.dev(q, t), pu.dev(k, t), pu.dev(v, t), pu.dev(qi), pu.dev(k.copy()), 1,
+                        density)
+    qn = pu.host(res.q_counts)[0]
+    assert (qn[5:] == 0).all() and (pu.host(res.k_counts) == 1).all()
+    pu.assert_attention_close(pu.host(res.o)[0], _dense(q[0], k[0], v[0], 1 / math.sqrt(d)), dtype)
+
+
+# --------------------------------------------------------------------------- full size, sampled
+@pytest.mark.slow
+def test_wan_layer_full_size_sampled():
+    """The 40-head Wan2.x layer (N = 75,600, C_q = 100, C_k = 500, rho = 0.10) in
+    the launch configuration the benchmark times; sampled checks per step."""
+    w = gen.WAN
+    L = gen.make_layer(w)
+    t = torch.bfloat16
+    q, k, v = pu.dev(L.q, t), pu.dev(L.k, t), pu.dev(L.v, t)
+    res = ear.ear_layer(q, k, v, pu.dev(L.q_init), pu.dev(L.k_init), w.iters, w.density,
+                        want_lse=True)
+    torch.cuda.synchronize()
+    assert ear.ear_get_device_status() == 0
+    s = pu.scale_of(w.d)
+    one = ear.ear_kmeans(k, pu.dev(L.k_init), 1)[1]
+    one = pu.host(one)
+    o = pu.host(res.o)
+    rng = np.random.default_rng(0)
+    for h in (0, w.heads - 1):
+        # k-means iteration 1 on sampled rows: assignment from the seeded init
+        rows = rng.choice(w.n, 2000, replace=False)
+        _, l_ref, _ = eo.kmeans(L.k[h][rows], L.k_init[h], 1)
+        pu.assert_labels_exact_or_tie(L.k[h][rows], L.k_init[h], one[h][rows], l_ref)
+        # permutation: stable and consistent with the labels
+        qlab, qperm = pu.host(res.q_labels)[h], pu.host(res.q_perm)[h]
+        p_ref, o_ref = eo.permute(qlab, w.c_q)
+        np.testing.assert_array_equal(qperm, p_ref)
+        np.testing.assert_array_equal(pu.host(res.q_offsets)[h], o_ref)
+        # probe with the GPU's centroids, route given the GPU's E
+        qn, kn = pu.host(res.q_counts)[h], pu.host(res.k_counts)[h]
+        klab = pu.host(res.k_labels)[h]
+        qc, kc = pu.host(res.q_centroids)[h], pu.host(res.k_centroids)[h]
+        e = pu.host(res.e)[h]
+        e_ref = eo.probe(qc, qn, L.k[h], klab, kc, kn, s)
+        np.testing.assert_allclose(e, e_ref, rtol=2e-5, atol=1e-7 * e_ref.max())
+        ex_ref, pairs_ref = eo.route(e.astype(np.float64), qn, kn, w.n, w.n, w.density)
+        np.testing.assert_array_equal(pu.host(res.exact)[h], ex_ref)
+        assert pu.host(res.exact_pairs)[h] == pairs_ref
+        # attention on sampled queries given the GPU's mask, labels and centroids
+        qi = rng.choice(w.n, 384, replace=False)
+        vm = eo.segment_mean(L.v[h], klab, w.c_k)
+        o_ref, _ = eo.attention(L.q[h][qi], L.k[h], L.v[h], qlab[qi], klab, kc, vm, kn, ex_ref, s)
+        pu.assert_attention_close(o[h][qi], o_ref, "bf16")
