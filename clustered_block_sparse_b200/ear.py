@@ -91,6 +91,31 @@ def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor]
     return perm, offsets, x_perm, mean
 
 
+def ear_permute_static(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor] = None,
+                       seg_mean: bool = False):
+    """ear_permute without a workspace, for callers that cannot allocate device
+    memory: the scratch lives in a fixed array inside libear (at most
+    EAR_PERMUTE_STATIC_MAX_BYTES).  Same results as ear_permute.  Calls that
+    overlap on the GPU share that array and race; run them one at a time."""
+    _need(labels, "labels")
+    bh, n = labels.shape
+    dev = labels.device
+    perm = torch.empty((bh, n), dtype=torch.int32, device=dev)
+    offsets = torch.empty((bh, n_clusters + 1), dtype=torch.int32, device=dev)
+    x_perm = mean = None
+    d, dt = 0, 0
+    if x is not None:
+        _need(x, "x")
+        d, dt = x.shape[2], _dtype(x)
+        x_perm = torch.empty_like(x)
+        if seg_mean:
+            mean = torch.empty((bh, n_clusters, d), dtype=torch.float32, device=dev)
+    N.check("ear_permute_static", N.lib().ear_permute_static(
+        _p(labels), bh, n, n_clusters, _p(perm), _p(offsets), _p(x), _p(x_perm), dt, d, _p(mean),
+        _stream(dev)))
+    return perm, offsets, x_perm, mean
+
+
 def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Optional[float] = None):
     """E[a,b] = sum_{j in b} (s q̄_a·k_j - s q̄_a·k̄_b)^2 (SVG-EAR §4.2). Returns E [BH,C_q,C_k] f32."""
     for t, nm in ((q_centroids, "q_centroids"), (q_counts, "q_counts"), (k_centroids, "k_centroids"),

@@ -134,6 +134,36 @@ EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int
                        void* stream);
 
 /*
+ * ear_permute_static - ear_permute for callers that cannot allocate device
+ * memory (the paper has no counterpart: this is a deployment variant).
+ *
+ * Some callers have no way to allocate scratch: a plugin whose host
+ * application owns every device buffer and passes in only inputs and
+ * outputs, or an embedded runtime with a fixed memory plan.  This entry point
+ * takes no workspace; its scratch is one fixed array of
+ * EAR_PERMUTE_STATIC_MAX_BYTES compiled into the library, which every GPU
+ * that loads the library keeps for the life of the process.
+ *   - Arguments, outputs and results are exactly those of ear_permute.
+ *   - The scratch needed is the one ear_workspace_bytes(EAR_OP_PERMUTE, ...)
+ *     reports; a problem needing more than EAR_PERMUTE_STATIC_MAX_BYTES is
+ *     rejected with EAR_ERR_WORKSPACE before anything runs.  (8 MiB holds,
+ *     e.g., 40 slices of 75,600 tokens in 500 clusters.)
+ *   - The first call on a device looks up the array's device address on
+ *     that device (the device must be current); make that first call before
+ *     any stream capture begins.
+ *   - No call allocates or frees memory (no cudaMalloc / cudaFree).
+ *   - Every call reuses the same array and leaves its contents behind; each
+ *     call clears what it needs zeroed.  Calls whose work overlaps on the
+ *     GPU (two streams, or two host threads, on one device) race on the
+ *     array: serialize them.
+ */
+#define EAR_PERMUTE_STATIC_MAX_BYTES (8u << 20)
+EAR_API ear_status ear_permute_static(const int32_t* labels, int64_t bh, int64_t n, int32_t c,
+                                      int32_t* perm, int32_t* offsets, const void* X,
+                                      void* X_perm, ear_dtype dtype, int32_t d, float* seg_mean,
+                                      void* stream);
+
+/*
  * Compensation-error probe (SVG-EAR §4.2 "Error estimation"; §1: query
  * centroids stand in for individual queries, O(C_q N_k d) work).
  *   q_centroids [BH][C_q][d] float     q̄_a
