@@ -251,37 +251,50 @@ ear_status simt_t(const AttnArgs& a, const int2* items, const int32_t* count, in
   return after_launch();
 }
 
+// Workspace: the unit list, plus bf16 copies of the key / value centroids
+// (rows padded to the tensor-core key chunk) for the tensor-core path.
 struct AtWs {
   int2* items;
   int32_t* count;
+  uint16_t* kc16;
+  uint16_t* vc16;
 };
 
-AtWs carve(Carver& cv, int64_t bh, int64_t n_q, int32_t c_q) {
+AtWs carve(Carver& cv, int64_t bh, int64_t n_q, int32_t d, int32_t c_q, int32_t c_k) {
   AtWs w;
   w.items = cv.take<int2>((size_t)bh * attn_items_per_slice(n_q, c_q));
   w.count = cv.take<int32_t>((size_t)bh);
+  const size_t cen = (size_t)bh * attention_tc_ck_pad(c_k) * d;
+  w.kc16 = cv.take<uint16_t>(cen);
+  w.vc16 = cv.take<uint16_t>(cen);
   return w;
 }
 
 }  // namespace
 
-size_t attention_workspace(int64_t bh, int64_t n_q, int32_t c_q, int32_t) {
+ear_status attention_plan(const int32_t* q_off, int64_t bh, int32_t c_q, int tile,
+                          int64_t max_items, int2* items, int32_t* count, cudaStream_t s) {
+  at_plan<<<(unsigned)bh, 1024, 0, s>>>(q_off, c_q, tile, max_items, items, count);
+  return after_launch();
+}
+
+size_t attention_workspace(int64_t bh, int64_t n_q, int32_t d, int32_t c_q, int32_t c_k) {
   Carver cv(nullptr);
-  carve(cv, bh, n_q, c_q);
+  carve(cv, bh, n_q, d, c_q, c_k);
   return cv.used;
 }
 
 ear_status attention_run(const AttnArgs& a, void* ws, cudaStream_t s) {
   Carver cv(ws);
-  AtWs w = carve(cv, a.bh, a.n_q, a.c_q);
+  AtWs w = carve(cv, a.bh, a.n_q, a.d, a.c_q, a.c_k);
+  if (a.dtype == EAR_BF16) {
+    const int64_t max_items = attention_tc_items_per_slice(a.n_q, a.c_q);
+    return attention_tc_run(a, w.items, w.count, max_items, w.kc16, w.vc16, s);
+  }
   const int64_t max_items = attn_items_per_slice(a.n_q, a.c_q);
-  at_plan<<<(unsigned)a.bh, 1024, 0, s>>>(a.q_off, a.c_q, kTile, max_items, w.items, w.count);
-  EAR_TRY(after_launch());
-  if (a.dtype == EAR_F32)
-    return a.d == 64 ? simt_t<float, 64>(a, w.items, w.count, max_items, s)
-                     : simt_t<float, 128>(a, w.items, w.count, max_items, s);
-  return a.d == 64 ? simt_t<uint16_t, 64>(a, w.items, w.count, max_items, s)
-                   : simt_t<uint16_t, 128>(a, w.items, w.count, max_items, s);
+  EAR_TRY(attention_plan(a.q_off, a.bh, a.c_q, kTile, max_items, w.items, w.count, s));
+  return a.d == 64 ? simt_t<float, 64>(a, w.items, w.count, max_items, s)
+                   : simt_t<float, 128>(a, w.items, w.count, max_items, s);
 }
 
 }  // namespace ear

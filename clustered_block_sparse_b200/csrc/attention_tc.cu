@@ -1,0 +1,562 @@
+// Block-sparse attention with linear compensation on the sm_100a tensor cores
+// (SVG-EAR §4.1 routing mask, §4.3 Linear Compensation), bf16 inputs, fp32
+// accumulation.
+//
+// One CTA = one unit of up to 256 permuted query rows of ONE query cluster a,
+// split in two 128-row tiles A and B (tcgen05.mma M = 128).  Both tiles walk
+// the same key chunks:
+//   * exact chunks: every key cluster b listed for a, in pieces of <= 128
+//     keys taken straight from the permuted K / V rows;
+//   * compensation chunks (EAR_COMPENSATE): the C_k key / value centroids in
+//     pieces of 128, with per-column bias log2|b| (weight |b|) and -inf for
+//     clusters that are exact for a or empty.
+// Warp roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, then K/V chunks into a 2-stage ring;
+//               computes the compensation bias of each centroid chunk.
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T into TMEM, then
+//               O_t += P_t V with P_t read from TMEM.  Issue order
+//               QK_A(c) QK_B(c) | PV_A(c) QK_A(c+1) PV_B(c) QK_B(c+1) | ...
+//               so one tile's softmax overlaps the other tile's MMAs.
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread
+//               per query row (= TMEM lane).  Online softmax in base 2; the
+//               running max is only moved (and O rescaled in TMEM) when it
+//               grows by more than 2^8, so most chunks skip the rescale.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512);
+// P_t (bf16 pairs) overwrites the first half of S_t.
+#include <mutex>
+
+#include "ear_internal.cuh"
+#include "sm100.cuh"
+
+namespace ear {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileRows = 128;
+constexpr int kTiles = 2;
+constexpr int kUnitRows = kTileRows * kTiles;
+constexpr int kChunk = 128;
+constexpr int kStages = 2;
+constexpr int kBoxRows = 32;
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;  // move the running max only when it grows by > 2^8
+
+// barrier slots
+constexpr int kBarKvFull = 0;   // + stage
+constexpr int kBarKvEmpty = 2;  // + stage
+constexpr int kBarQFull = 4;
+constexpr int kBarSFull = 5;    // + tile
+constexpr int kBarPFull = 7;    // + tile
+constexpr int kBarODone = 9;    // + tile
+constexpr int kBarDrain = 11;   // teardown: every MMA issued has finished
+constexpr int kNumBars = 12;
+
+template <int D>
+struct Layout {
+  static constexpr int kHalfBytes = kTileRows * 128;  // 128 rows x 64 bf16
+  static constexpr int kTileBytes = kHalfBytes * (D / 64);
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTiles * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBias = kV + kStages * kTileBytes;
+  static constexpr int kBar = kBias + kStages * kChunk * 4;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
+};
+
+struct TcParams {
+  const int32_t* q_off;
+  const int32_t* k_off;
+  const int32_t* q_perm;
+  const uint8_t* exact;
+  const int32_t* blk_off;
+  const int32_t* blk_list;
+  const int2* items;
+  const int32_t* count;
+  int64_t max_items;
+  int64_t Nq, Nk;
+  int Cq, Ck, Ck_pad;
+  float qk_scale;  // scale * log2(e)
+  int compensate;
+  uint16_t* O;
+  float* lse;
+  int* status;
+};
+
+// The chunk sequence of one unit; every role walks its own copy.
+struct Chunks {
+  const int32_t* list;
+  const int32_t* koff;
+  int32_t e, e1, pos, end;
+  int32_t comp_next, Ck, Nk;
+  int compensate;
+  int* status;
+
+  __device__ void init(const TcParams& p, int64_t h, int a) {
+    const int32_t* bo = p.blk_off + h * (int64_t)(p.Cq + 1);
+    list = p.blk_list + h * (int64_t)p.Cq * p.Ck;
+    koff = p.k_off + h * (int64_t)(p.Ck + 1);
+    e = bo[a];
+    e1 = bo[a + 1];
+    pos = end = 0;
+    comp_next = 0;
+    Ck = p.Ck;
+    Nk = (int32_t)p.Nk;
+    compensate = p.compensate;
+    status = p.status;
+  }
+  // row: first key row within the slice (exact) or first centroid (compensation);
+  // comp = whether this is a centroid chunk.
+  __device__ bool next(int32_t& row, int& nv, bool& comp) {
+    while (pos >= end && e < e1) {
+      const int b = list[e++];
+      if (b < 0 || b >= Ck) {
+        latch(status, EAR_ERR_DEVICE);
+        continue;
+      }
+      pos = koff[b];
+      end = koff[b + 1];
+      if (pos < 0 || end > Nk || end < pos) {
+        latch(status, EAR_ERR_DEVICE);
+        pos = end = 0;
+      }
+    }
+    if (pos < end) {
+      row = pos;
+      nv = min(kChunk, end - pos);
+      pos += nv;
+      comp = false;
+      return true;
+    }
+    if (compensate && comp_next < Ck) {
+      row = comp_next;
+      nv = min(kChunk, Ck - comp_next);
+      comp_next += kChunk;
+      comp = true;
+      return true;
+    }
+    return false;
+  }
+};
+
+__device__ __forceinline__ int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+      const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int64_t h = blockIdx.y;
+  const int64_t slot = blockIdx.x;
+  if (slot >= p.count[h]) return;
+  const int2 item = p.items[h * p.max_items + slot];
+  const int a = item.x;
+  const int32_t row0 = item.y;
+  const int32_t qend = p.q_off[h * (int64_t)(p.Cq + 1) + a + 1];
+  if (row0 < 0 || qend > p.Nq || row0 >= qend) {
+    if (threadIdx.x == 0) latch(p.status, EAR_ERR_DEVICE);
+    return;
+  }
+  const int rows_t[2] = {min(kTileRows, qend - row0), max(0, min(kTileRows, qend - row0 - kTileRows))};
+  const int ntiles = rows_t[1] > 0 ? 2 : 1;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* bias = reinterpret_cast<float*>(smem + L::kBias);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[kBarKvFull + s], 1);
+      mbar_init(&bars[kBarKvEmpty + s], 1);
+    }
+    mbar_init(&bars[kBarQFull], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&bars[kBarSFull + t], 1);
+      mbar_init(&bars[kBarPFull + t], kTileRows);
+      mbar_init(&bars[kBarODone + t], 1);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const uint8_t* exact_row = p.exact + (h * p.Cq + a) * (int64_t)p.Ck;
+    const int32_t* koff = p.k_off + h * (int64_t)(p.Ck + 1);
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars[kBarQFull], ntiles * L::kTileBytes);
+      for (int t = 0; t < ntiles; ++t)
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d(smem + L::kQ + t * L::kTileBytes + hf * L::kHalfBytes, &tmQ,
+                      &bars[kBarQFull], 64 * hf, (int32_t)(h * p.Nq) + row0 + kTileRows * t);
+    }
+    Chunks it;
+    it.init(p, h, a);
+    int32_t row;
+    int nv;
+    bool comp;
+    int issued = 0;
+    for (int c = 0; it.next(row, nv, comp); ++c) {
+      const int s = c % kStages;
+      if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
+        break;
+      issued = c + 1;
+      if (comp) {
+        for (int j = lane; j < kChunk; j += 32) {
+          float bv = -INFINITY;
+          if (j < nv) {
+            const int b = row + j;
+            const int32_t cnt = koff[b + 1] - koff[b];
+            if (!exact_row[b] && cnt > 0) bv = __log2f((float)cnt);
+          }
+          bias[s * kChunk + j] = bv;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int npad = round_up(nv, kBoxRows);
+        mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * npad * D * 2);
+        const CUtensorMap* mk = comp ? &tmKc : &tmK;
+        const CUtensorMap* mv = comp ? &tmVc : &tmV;
+        const int32_t grow = comp ? (int32_t)(h * p.Ck_pad) + row : (int32_t)(h * p.Nk) + row;
+        uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
+        uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
+        for (int r = 0; r < npad; r += kBoxRows)
+          for (int hf = 0; hf < D / 64; ++hf) {
+            tma_load_2d(kdst + hf * L::kHalfBytes + r * 128, mk, &bars[kBarKvFull + s], 64 * hf,
+                        grow + r);
+            tma_load_2d(vdst + hf * L::kHalfBytes + r * 128, mv, &bars[kBarKvFull + s], 64 * hf,
+                        grow + r);
+          }
+      }
+      __syncwarp();
+    }
+    // Teardown after an abort: let the loads already issued land before the
+    // CTA exits (a no-op when the consumers saw every chunk).
+    if (*abort) {
+      mbar_wait_drain(&bars[kBarQFull], 0);
+      for (int c = issued - 1; c >= 0 && c >= issued - kStages; --c)
+        mbar_wait_drain(&bars[kBarKvFull + c % kStages], (c / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16(128, D, true);
+      auto issue_qk = [&](int t, int s, int n) {
+        const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
+        const uint32_t qb = smem_u32(smem + L::kQ + t * L::kTileBytes);
+        const uint32_t kb = smem_u32(smem + L::kK + s * L::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * L::kHalfBytes + (kk % 4) * 32;
+          mma_ss(tmem + kTileRows * t, desc_sw128(qb + off, 16, 1024),
+                 desc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, int n, bool first) {
+        const uint32_t vb = smem_u32(smem + L::kV + s * L::kTileBytes);
+        for (int kk = 0; kk < n / 16; ++kk)
+          mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kk * 8,
+                 desc_sw128(vb + kk * 2048, L::kHalfBytes, 1024), idesc_pv,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      Chunks it;
+      it.init(p, h, a);
+      int32_t row;
+      int nv;
+      bool comp;
+      bool have = it.next(row, nv, comp);
+      int n_cur = round_up(nv, 16);
+      bool ok = mbar_wait(&bars[kBarQFull], 0, abort);
+      if (ok && have) {
+        ok = mbar_wait(&bars[kBarKvFull + 0], 0, abort);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < ntiles; ++t) {
+            issue_qk(t, 0, n_cur);
+            mma_commit(&bars[kBarSFull + t]);
+          }
+        }
+      }
+      for (int c = 0; ok && have; ++c) {
+        const int s = c % kStages;
+        const int s2 = (c + 1) % kStages;
+        int32_t row2;
+        int nv2;
+        bool comp2;
+        const bool have2 = it.next(row2, nv2, comp2);
+        const int n_nxt = round_up(nv2, 16);
+        for (int t = 0; t < ntiles && ok; ++t) {
+          ok = mbar_wait(&bars[kBarPFull + t], c & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, s, n_cur, c == 0);
+          mma_commit(&bars[kBarODone + t]);
+          if (t == ntiles - 1) mma_commit(&bars[kBarKvEmpty + s]);
+          if (have2) {
+            if (t == 0) {
+              ok = mbar_wait(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_qk(t, s2, n_nxt);
+            mma_commit(&bars[kBarSFull + t]);
+          }
+        }
+        have = have2;
+        n_cur = n_nxt;
+      }
+      // every MMA issued above has finished before TMEM is released
+      mma_commit(&bars[kBarDrain]);
+      mbar_wait_drain(&bars[kBarDrain], 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax
+    const int t = (warp - 4) / 4;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // row within the tile = TMEM lane
+    if (t < ntiles) {
+      const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_bits + kTileRows * t;
+      const uint32_t tO = tmem + lane_bits + 256 + kTileRows * t;
+      float m = -INFINITY, l = 0.f;
+      Chunks it;
+      it.init(p, h, a);
+      int32_t row;
+      int nv;
+      bool comp;
+      int c = 0;
+      bool ok = true;
+      uint32_t v[32];
+      for (; it.next(row, nv, comp); ++c) {
+        const int s = c % kStages;
+        ok = mbar_wait(&bars[kBarSFull + t], c & 1, abort);
+        if (ok && comp) ok = mbar_wait(&bars[kBarKvFull + s], (c / kStages) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const float* bs = bias + s * kChunk;
+        const int ng = (nv + 31) / 32;
+        float mx = -INFINITY;
+        for (int g = 0; g < ng; ++g) {
+          tmem_ld32(tS + 32 * g, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = 32 * g + j;
+            float z = __uint_as_float(v[j]) * p.qk_scale + (comp ? bs[col] : 0.f);
+            z = col < nv ? z : -INFINITY;
+            mx = fmaxf(mx, z);
+          }
+        }
+        float m_use = m, corr = 1.f;
+        bool resc = false;
+        if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
+          if (m != -INFINITY) {
+            resc = true;
+            corr = ex2(m - mx);
+          }
+          m_use = mx;
+        }
+        l *= corr;
+        for (int g = 0; g < ng; ++g) {
+          tmem_ld32(tS + 32 * g, v);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int col = 32 * g + j;
+            float z0 = __uint_as_float(v[j]) * p.qk_scale + (comp ? bs[col] : 0.f);
+            float z1 = __uint_as_float(v[j + 1]) * p.qk_scale + (comp ? bs[col + 1] : 0.f);
+            const float p0 = (col < nv && m_use != -INFINITY) ? ex2(z0 - m_use) : 0.f;
+            const float p1 = (col + 1 < nv && m_use != -INFINITY) ? ex2(z1 - m_use) : 0.f;
+            l += p0 + p1;
+            pk[j / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * g, pk);
+        }
+        tmem_st_wait();
+        if (__any_sync(0xffffffffu, resc)) {
+          ok = mbar_wait(&bars[kBarODone + t], (c - 1) & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          for (int g = 0; g < D / 32; ++g) {
+            tmem_ld32(tO + 32 * g, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * corr);
+            tmem_st32(tO + 32 * g, v);
+          }
+          tmem_st_wait();
+        }
+        m = m_use;
+        tc_fence_before();
+        mbar_arrive(&bars[kBarPFull + t]);
+      }
+      // epilogue: O / l written at the queries' original positions
+      const int32_t prow = row0 + kTileRows * t + r;
+      const int32_t orig = r < rows_t[t] ? p.q_perm[h * p.Nq + prow] : -1;
+      const bool valid = orig >= 0 && orig < p.Nq;
+      if (r < rows_t[t] && !valid) latch(p.status, EAR_ERR_DEVICE);
+      const bool have_o = ok && c > 0 && mbar_wait(&bars[kBarODone + t], (c - 1) & 1, abort);
+      if (have_o) tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint16_t* orow = p.O + ((int64_t)h * p.Nq + (valid ? orig : 0)) * D;
+      for (int g = 0; g < D / 32; ++g) {
+        if (have_o) {
+          tmem_ld32(tO + 32 * g, v);
+          tmem_ld_wait();
+        }
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2)
+            pk[j / 2] = have_o ? pack_bf16x2(__uint_as_float(v[j]) * inv,
+                                             __uint_as_float(v[j + 1]) * inv)
+                               : 0u;
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * g);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[h * p.Nq + orig] = (have_o && l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort) latch(p.status, EAR_ERR_TIMEOUT);
+}
+
+__global__ void at_centroids_bf16(const float* __restrict__ kc, const float* __restrict__ vc,
+                                  uint16_t* __restrict__ kc16, uint16_t* __restrict__ vc16,
+                                  int Ck, int Ck_pad, int D, int64_t total) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const int64_t hc = e / D;
+  const int k = (int)(e % D);
+  const int64_t h = hc / Ck_pad;
+  const int c = (int)(hc % Ck_pad);
+  const bool ok = c < Ck;
+  kc16[e] = ok ? f32_to_bf16(kc[(h * Ck + c) * D + k]) : 0;
+  vc16[e] = ok ? f32_to_bf16(vc[(h * Ck + c) * D + k]) : 0;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows][d], 64-column x box_rows boxes, 128-byte swizzle,
+// zero fill past the last row.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_items,
+                uint16_t* kc16, uint16_t* vc16, int ck_pad, cudaStream_t s) {
+  using L = Layout<D>;
+  const int64_t total = a.bh * (int64_t)ck_pad * D;
+  at_centroids_bf16<<<(unsigned)ceil_div(total, 256), 256, 0, s>>>(a.k_cent, a.v_cent, kc16, vc16,
+                                                                   a.c_k, ck_pad, D, total);
+  EAR_TRY(after_launch());
+  CUtensorMap mq, mk, mv, mkc, mvc;
+  if (!make_map(&mq, a.Q, a.bh * a.n_q, D, kTileRows) ||
+      !make_map(&mk, a.K, a.bh * a.n_k, D, kBoxRows) ||
+      !make_map(&mv, a.V, a.bh * a.n_k, D, kBoxRows) ||
+      !make_map(&mkc, kc16, a.bh * ck_pad, D, kBoxRows) ||
+      !make_map(&mvc, vc16, a.bh * ck_pad, D, kBoxRows))
+    return EAR_ERR_CUDA;
+  TcParams p;
+  p.q_off = a.q_off;
+  p.k_off = a.k_off;
+  p.q_perm = a.q_perm;
+  p.exact = a.exact;
+  p.blk_off = a.blk_off;
+  p.blk_list = a.blk_list;
+  p.items = items;
+  p.count = count;
+  p.max_items = max_items;
+  p.Nq = a.n_q;
+  p.Nk = a.n_k;
+  p.Cq = a.c_q;
+  p.Ck = a.c_k;
+  p.Ck_pad = ck_pad;
+  p.qk_scale = a.scale * kLog2e;
+  p.compensate = a.flags & EAR_COMPENSATE;
+  p.O = static_cast<uint16_t*>(a.O);
+  p.lse = a.lse;
+  p.status = device_status_word();
+  EAR_CUDA(cudaFuncSetAttribute(at_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  const dim3 grid((unsigned)max_items, (unsigned)a.bh);
+  at_tc<D><<<grid, kThreads, L::kBytes, s>>>(mq, mk, mv, mkc, mvc, p);
+  return after_launch();
+}
+
+}  // namespace
+
+int64_t attention_tc_ck_pad(int32_t c_k) { return ceil_div(c_k, kChunk) * kChunk; }
+
+int64_t attention_tc_items_per_slice(int64_t n_q, int32_t c_q) {
+  return ceil_div(n_q, kUnitRows) + c_q;
+}
+
+ear_status attention_tc_run(const AttnArgs& a, int2* items, int32_t* count, int64_t max_items,
+                            uint16_t* kc16, uint16_t* vc16, cudaStream_t s) {
+  EAR_TRY(attention_plan(a.q_off, a.bh, a.c_q, kUnitRows, max_items, items, count, s));
+  const int ck_pad = (int)attention_tc_ck_pad(a.c_k);
+  return a.d == 64 ? tc_t<64>(a, items, count, max_items, kc16, vc16, ck_pad, s)
+                   : tc_t<128>(a, items, count, max_items, kc16, vc16, ck_pad, s);
+}
+
+}  // namespace ear

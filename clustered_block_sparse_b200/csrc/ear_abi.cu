@@ -81,7 +81,7 @@ ear_status ear_workspace_bytes(ear_op op, int64_t bh, int64_t n_q, int64_t n_k, 
     case EAR_OP_PERMUTE: *bytes = ear::permute_workspace(bh, n_q, c_q); return EAR_OK;
     case EAR_OP_PROBE: *bytes = ear::probe_workspace(bh, n_k, d, c_q, c_k); return EAR_OK;
     case EAR_OP_ROUTE: *bytes = ear::route_workspace(bh, c_q, c_k); return EAR_OK;
-    case EAR_OP_ATTENTION: *bytes = ear::attention_workspace(bh, n_q, c_q, c_k); return EAR_OK;
+    case EAR_OP_ATTENTION: *bytes = ear::attention_workspace(bh, n_q, d, c_q, c_k); return EAR_OK;
   }
   return EAR_ERR_ARG;
 }
@@ -181,7 +181,7 @@ ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_p
     return EAR_ERR_ARG;
   if (lse != nullptr && !aligned16(lse)) return EAR_ERR_ARG;
   if (!ok_d(d) || c_q > kMaxC || c_k > kMaxC || bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
-  EAR_TRY(check_ws(ws, ws_bytes, ear::attention_workspace(bh, n_q, c_q, c_k)));
+  EAR_TRY(check_ws(ws, ws_bytes, ear::attention_workspace(bh, n_q, d, c_q, c_k)));
   if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
   ear::AttnArgs a{Q_perm, K_perm, V_perm, dtype, q_offsets, k_offsets, q_perm, k_centroids,
                   v_centroids, exact, blk_offsets, blk_list, bh, n_q, n_k, d, c_q, c_k, scale,

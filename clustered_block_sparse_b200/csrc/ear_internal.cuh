@@ -91,8 +91,16 @@ struct AttnArgs {
   void* O;
   float* lse;
 };
-size_t attention_workspace(int64_t bh, int64_t n_q, int32_t c_q, int32_t c_k);
+size_t attention_workspace(int64_t bh, int64_t n_q, int32_t d, int32_t c_q, int32_t c_k);
 ear_status attention_run(const AttnArgs& a, void* ws, cudaStream_t s);
+// Query units of `tile` rows that never straddle two query clusters.
+ear_status attention_plan(const int32_t* q_off, int64_t bh, int32_t c_q, int tile,
+                          int64_t max_items, int2* items, int32_t* count, cudaStream_t s);
+// Tensor-core path (bf16): centroid rows padded to a multiple of the key chunk.
+int64_t attention_tc_ck_pad(int32_t c_k);
+int64_t attention_tc_items_per_slice(int64_t n_q, int32_t c_q);
+ear_status attention_tc_run(const AttnArgs& a, int2* items, int32_t* count, int64_t max_items,
+                            uint16_t* kc16, uint16_t* vc16, cudaStream_t s);
 
 }  // namespace ear
 
