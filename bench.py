@@ -399,12 +399,17 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ear", "reference"), default="ear")
     ap.add_argument("--workload", choices=tuple(WORKLOADS), default="wan")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the head count (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.heads is not None and args.heads != w.heads:
+        w = w.with_(heads=args.heads, name=f"{w.name.split('-')[0]}-shape-{args.heads}head-"
+                    f"N{w.n}-d{w.d}-{w.dtype}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ear(args, w)

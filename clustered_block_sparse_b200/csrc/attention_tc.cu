@@ -352,8 +352,8 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
       uint32_t v[32];
       for (; it.next(row, nv, comp); ++c) {
         const int s = c % kStages;
-        ok = mbar_wait(&bars[kBarSFull + t], c & 1, abort);
-        if (ok && comp) ok = mbar_wait(&bars[kBarKvFull + s], (c / kStages) & 1, abort);
+        ok = mbar_wait_warp(&bars[kBarSFull + t], c & 1, abort);
+        if (ok && comp) ok = mbar_wait_warp(&bars[kBarKvFull + s], (c / kStages) & 1, abort);
         if (!ok) break;
         tc_fence_after();
         const float* bs = bias + s * kChunk;
@@ -398,7 +398,7 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
         }
         tmem_st_wait();
         if (__any_sync(0xffffffffu, resc)) {
-          ok = mbar_wait(&bars[kBarODone + t], (c - 1) & 1, abort);
+          ok = mbar_wait_warp(&bars[kBarODone + t], (c - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
           for (int g = 0; g < D / 32; ++g) {
@@ -419,7 +419,7 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
       const int32_t orig = r < rows_t[t] ? p.q_perm[h * p.Nq + prow] : -1;
       const bool valid = orig >= 0 && orig < p.Nq;
       if (r < rows_t[t] && !valid) latch(p.status, EAR_ERR_DEVICE);
-      const bool have_o = ok && c > 0 && mbar_wait(&bars[kBarODone + t], (c - 1) & 1, abort);
+      const bool have_o = ok && c > 0 && mbar_wait_warp(&bars[kBarODone + t], (c - 1) & 1, abort);
       if (have_o) tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint16_t* orow = p.O + ((int64_t)h * p.Nq + (valid ? orig : 0)) * D;

@@ -55,6 +55,12 @@ ear_status kmeans_run(const void* X, ear_dtype dt, int64_t bh, int64_t n, int32_
                       int32_t iters, const float* init, float* cent, int32_t* labels,
                       int32_t* counts, void* ws, cudaStream_t s);
 
+bool kmeans_tc_supported(ear_dtype dt, int32_t d, int32_t c);
+size_t kmeans_tc_workspace(int64_t bh, int64_t n, int32_t d, int32_t c);
+ear_status kmeans_tc_run(const void* X, int64_t bh, int64_t n, int32_t d, int32_t c,
+                         int32_t iters, const float* init, float* cent, int32_t* labels,
+                         int32_t* counts, void* ws, cudaStream_t s);
+
 size_t permute_workspace(int64_t bh, int64_t n, int32_t c);
 ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, int32_t* perm,
                        int32_t* offsets, const void* X, void* X_perm, ear_dtype dt, int32_t d,

@@ -12,6 +12,8 @@
 //    the exact fp64 argmin, ties to the lowest index.
 //  * km_update: member sums with vector fp32 atomics, counts with int atomics.
 //  * km_finalize: centroid = sum / count; an empty cluster keeps its centroid.
+#include <algorithm>
+
 #include "ear_internal.cuh"
 
 namespace ear {
@@ -255,15 +257,21 @@ ear_status run_t(const T* X, int64_t bh, int64_t n, int32_t c, int32_t iters, co
 
 }  // namespace
 
+// The tensor-core path serves bf16 inputs with at most 512 centroids; the
+// workspace covers whichever path the dtype selects.
 size_t kmeans_workspace(int64_t bh, int64_t n, int32_t d, int32_t c) {
   Carver cv(nullptr);
   carve(cv, bh, n, d, c);
-  return cv.used;
+  size_t bytes = cv.used;
+  if (kmeans_tc_supported(EAR_BF16, d, c)) bytes = std::max(bytes, kmeans_tc_workspace(bh, n, d, c));
+  return bytes;
 }
 
 ear_status kmeans_run(const void* X, ear_dtype dt, int64_t bh, int64_t n, int32_t d, int32_t c,
                       int32_t iters, const float* init, float* cent, int32_t* labels,
                       int32_t* counts, void* ws, cudaStream_t s) {
+  if (kmeans_tc_supported(dt, d, c))
+    return kmeans_tc_run(X, bh, n, d, c, iters, init, cent, labels, counts, ws, s);
   if (dt == EAR_F32) {
     if (d == 64)
       return run_t<float, 64>((const float*)X, bh, n, c, iters, init, cent, labels, counts, ws, s);

@@ -1,0 +1,830 @@
+// Lloyd k-means on the sm_100a tensor cores (SVG-EAR §4.1: Q and K are
+// clustered and each token is represented by the mean token of its cluster).
+// Used for bf16 inputs with C <= 512 centroids; labels are exact.
+//
+// Per call:
+//   km_xprep     X (bf16) -> fp16 copy Xh plus ||x|| per row.  A row with a
+//                value beyond the fp16 range gets ||x|| = +inf (always re-decided).
+//   km_cprep     centroids -> fp16 copy, fp32 ||c||^2 (+inf on padding
+//                columns), per-slice max ||c||.
+// Per iteration:
+//   km_tc        one CTA = up to 8 tiles of 128 rows of one slice.  The
+//                slice's fp16 centroids stay in shared memory; a TMA warp
+//                streams X tiles, one thread issues tcgen05.mma
+//                (S = X C^T, fp32, 256-column chunks, two TMEM buffers) and
+//                two epilogue warpgroups scan each chunk (alternate 32-column
+//                groups) twice: pass 1 takes the minimum of
+//                d~_c = ||c||^2 - 2 x.c^, pass 2 collects every column within
+//                the rounding margin of the running minimum.  One candidate
+//                = a certain label; 2-4 candidates go to an fp64 decision
+//                among them; more (or a row / centroid without an exact fp16
+//                copy) go to a full fp64 decision.  Certain rows whose label
+//                changed are listed as moves.
+//   km_pick64    fp64 distances of the 2-4 candidates of a listed row, in the
+//                order sum_k (x_k - c_k)^2 k = 0..d-1 (ties to the lowest
+//                index), then the row's move.
+//   km_refine64  the same over all C centroids for the rows that need it.
+//   km_moves     sums[new] += x, sums[old] -= x, counts likewise (vector fp32
+//                atomics): after the first iteration only moved rows cost work.
+//   km_finalize  centroid = sum / count (empty clusters keep theirs), and the
+//                fp16 copy / norms / max norm for the next iteration.
+//
+// Rounding bound of the approximate distance d~_c = ||c||^2 - 2 x.c^ (c^ =
+// fp16(c), products exact, fp32 accumulation over d terms, ||c||^2 in fp32):
+//   |d~_c - (||x - c||^2 - ||x||^2)| <= a ||x|| Cmax + b Cmax^2
+//                                            + s (||x|| + Cmax)
+//   a = 2 (2^-11 + (d + 1) 2^-23)(1 + 2^-11) (1 + 2^-20),  b = 2^-16,
+//   s = 2 sqrt(d) 2^-25 (centroid or x values in the fp16 subnormal range
+//   round with absolute error <= 2^-25)
+// (Cauchy-Schwarz turns sum |x_k c_k| into ||x|| ||c||, Cmax = max ||c||.)
+// A centroid value beyond the fp16 range makes its slice fall back to fp64
+// for every row; an X row with a value beyond it always does.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "ear_internal.cuh"
+#include "sm100.cuh"
+
+namespace ear {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileRows = 128;
+constexpr int kTilesPerCta = 16;
+constexpr int kColChunk = 256;
+constexpr int kMaxCPad = 512;
+constexpr int kXStages = 2;
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 epilogue
+
+constexpr int kBarXFull = 0;    // + stage
+constexpr int kBarXEmpty = 2;   // + stage
+constexpr int kBarCFull = 4;
+constexpr int kBarTmFull = 5;   // + buffer
+constexpr int kBarTmEmpty = 7;  // + buffer
+constexpr int kBarDrain = 9;
+constexpr int kNumBars = 10;
+
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t m, uint32_t n) {
+  return (1u << 4) | ((n >> 3) << 17) | ((m >> 4) << 24);  // D f32, A/B f16, K-major
+}
+
+template <int D>
+struct KLayout {
+  static constexpr int kXHalf = kTileRows * 128;
+  static constexpr int kXTile = kXHalf * (D / 64);
+  static constexpr int kCHalf = kMaxCPad * 128;
+  static constexpr int kC = 0;
+  static constexpr int kX = kC + kCHalf * (D / 64);
+  static constexpr int kNorm = kX + kXStages * kXTile;
+  static constexpr int kXchg = kNorm + kMaxCPad * 4;   // [2][128] x 10 words
+  static constexpr int kBar = kXchg + 2 * kTileRows * 40;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16 + 1024;
+};
+
+struct Move {
+  int64_t row;
+  int32_t from;
+  int32_t to;
+};
+
+struct Pick {
+  int64_t row;
+  int32_t n;
+  int32_t cand[4];
+  int32_t pad;
+};
+
+struct KmTcParams {
+  const float* xnorm;       // [BH*N]
+  const float* cnorm;       // [BH*C_pad]
+  const float* cmax;        // [BH]
+  const int* cbad;          // [BH] a centroid of the slice has no finite fp16 copy
+  int32_t* labels;          // [BH*N]
+  int64_t* refine_rows;     // rows for the full fp64 decision
+  unsigned long long* refine_count;
+  struct Pick* picks;       // rows with 2-4 candidates
+  unsigned long long* pick_count;
+  Move* moves;
+  unsigned long long* move_count;
+  int64_t N;
+  int C, C_pad, first;
+  int c_box;  // rows per centroid TMA box (min(256, C_pad))
+  float a_coef, b_coef, s_coef;
+};
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Appends one entry per active lane with a single atomic per warp.
+__device__ __forceinline__ unsigned long long warp_append(unsigned long long* counter, bool want) {
+  const unsigned mask = __ballot_sync(0xffffffffu, want);
+  const int lane = threadIdx.x & 31;
+  unsigned long long base = 0;
+  const int leader = mask ? __ffs(mask) - 1 : 0;
+  if (mask && lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(mask));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  return base + __popc(mask & ((1u << lane) - 1u));
+}
+
+// min over 32 columns of d~ = cn - 2 v, four independent chains
+__device__ __forceinline__ float group_min(const uint32_t (&v)[32], const float* cn) {
+  const unsigned long long m2 = 0xC0000000C0000000ull;  // (-2.f, -2.f)
+  const unsigned long long* c2 = reinterpret_cast<const unsigned long long*>(cn);
+  float m[4] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000),
+                __int_as_float(0x7f800000), __int_as_float(0x7f800000)};
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    const unsigned long long vv = (unsigned long long)v[k] | ((unsigned long long)v[k + 1] << 32);
+    unsigned long long dd;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dd) : "l"(vv), "l"(m2), "l"(c2[k / 2]));
+    const int a = (k / 2) & 1;
+    m[2 * a] = fminf(m[2 * a], __uint_as_float((uint32_t)dd));
+    m[2 * a + 1] = fminf(m[2 * a + 1], __uint_as_float((uint32_t)(dd >> 32)));
+  }
+  return fminf(fminf(m[0], m[1]), fminf(m[2], m[3]));
+}
+
+// bit k set where d~ of column k is <= thr
+__device__ __forceinline__ uint32_t group_hits(const uint32_t (&v)[32], const float* cn, float thr) {
+  uint32_t hit = 0;
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    hit |= (fmaf(-2.f, __uint_as_float(v[k]), cn[k]) <= thr ? 1u : 0u) << k;
+  return hit;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
+      const KmTcParams p, int* status) {
+  using L = KLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int64_t h = blockIdx.y;
+  const int64_t tile0 = (int64_t)blockIdx.x * kTilesPerCta;
+  const int64_t ntiles_slice = (p.N + kTileRows - 1) / kTileRows;
+  const int64_t left = ntiles_slice - tile0;
+  const int ntiles = (int)(left < kTilesPerCta ? left : kTilesPerCta);
+  if (ntiles <= 0) return;
+  const int nch = (p.C_pad + kColChunk - 1) / kColChunk;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* cn = reinterpret_cast<float*>(smem + L::kNorm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(&bars[kBarXFull + s], 1);
+      mbar_init(&bars[kBarXEmpty + s], 1);
+    }
+    mbar_init(&bars[kBarCFull], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kBarTmFull + b], 1);
+      mbar_init(&bars[kBarTmEmpty + b], 256);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  for (int c = threadIdx.x; c < kMaxCPad; c += kThreads)
+    cn[c] = c < p.C_pad ? p.cnorm[h * p.C_pad + c] : __int_as_float(0x7f800000);
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmC);
+      const int nbox = (p.C_pad + p.c_box - 1) / p.c_box;  // whole boxes land, padding included
+      mbar_arrive_expect_tx(&bars[kBarCFull], nbox * p.c_box * D * 2);
+      for (int r = 0; r < nbox * p.c_box; r += p.c_box)
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d(smem + L::kC + hf * L::kCHalf + r * 128, &tmC, &bars[kBarCFull], 64 * hf,
+                      (int32_t)(h * p.C_pad) + r);
+    }
+    int issued = 0;
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kXStages;
+      if (t >= kXStages && !mbar_wait(&bars[kBarXEmpty + s], ((t / kXStages) - 1) & 1, abort))
+        break;
+      issued = t + 1;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[kBarXFull + s], L::kXTile);
+        const int32_t row = (int32_t)(h * p.N + (tile0 + t) * kTileRows);
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d(smem + L::kX + s * L::kXTile + hf * L::kXHalf, &tmX, &bars[kBarXFull + s],
+                      64 * hf, row);
+      }
+      __syncwarp();
+    }
+    if (*abort) {
+      mbar_wait_drain(&bars[kBarCFull], 0);
+      for (int t = issued - 1; t >= 0 && t >= issued - kXStages; --t)
+        mbar_wait_drain(&bars[kBarXFull + t % kXStages], (t / kXStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&bars[kBarCFull], 0, abort);
+      const uint32_t cb = smem_u32(smem + L::kC);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int s = t % kXStages;
+        ok = mbar_wait(&bars[kBarXFull + s], (t / kXStages) & 1, abort);
+        if (!ok) break;
+        const uint32_t xb = smem_u32(smem + L::kX + s * L::kXTile);
+        for (int j = 0; j < nch; ++j) {
+          const int i = t * nch + j, b = i & 1;
+          if (i >= 2) {
+            ok = mbar_wait(&bars[kBarTmEmpty + b], ((i >> 1) - 1) & 1, abort);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const int n = min(kColChunk, p.C_pad - j * kColChunk);
+          const uint32_t idesc = idesc_f16(128, (uint32_t)n);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t xo = (kk / 4) * L::kXHalf + (kk % 4) * 32;
+            const uint32_t co = (kk / 4) * L::kCHalf + j * kColChunk * 128 + (kk % 4) * 32;
+            mma_ss(tmem + b * kColChunk, desc_sw128(xb + xo, 16, 1024),
+                   desc_sw128(cb + co, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars[kBarTmFull + b]);
+        }
+        if (ok) mma_commit(&bars[kBarXEmpty + s]);
+      }
+      mma_commit(&bars[kBarDrain]);
+      mbar_wait_drain(&bars[kBarDrain], 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int w = (warp - 4) >> 2;       // warpgroup: column groups g with g % 2 == w
+    const int q = warp & 3;
+    const int r = q * 32 + lane;         // row within the tile = TMEM lane
+    const uint32_t lane_bits = (uint32_t)(q * 32) << 16;
+    // exchange [2 tiles][128 rows]: running min, count, 4 candidates, 4 distances
+    float* xrun = reinterpret_cast<float*>(smem + L::kXchg);
+    int* xcnt = reinterpret_cast<int*>(xrun + 2 * kTileRows);
+    int* xcand = xcnt + 2 * kTileRows;                                    // [.][4]
+    float* xdist = reinterpret_cast<float*>(xcand + 8 * kTileRows);       // [.][4]
+    const float inf = __int_as_float(0x7f800000);
+    const float cmax = p.cmax[h];
+    const bool cbad = p.cbad[h] != 0;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int64_t row = (tile0 + t) * kTileRows + r;
+      const bool valid = row < p.N;
+      const int64_t g = h * p.N + row;
+      const float xn = valid ? p.xnorm[g] : 0.f;
+      const float margin =
+          2.f * (p.a_coef * xn * cmax + p.b_coef * cmax * cmax + p.s_coef * (xn + cmax));
+      float run = inf;
+      int nc = 0, c0 = -1, c1 = -1, c2 = -1, c3 = -1;
+      float d0 = inf, d1 = inf, d2 = inf, d3 = inf;
+      for (int j = 0; j < nch && ok; ++j) {
+        const int i = t * nch + j, b = i & 1;
+        ok = mbar_wait_warp(&bars[kBarTmFull + b], (i >> 1) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const int n = min(kColChunk, p.C_pad - j * kColChunk);
+        const uint32_t tbuf = tmem + lane_bits + b * kColChunk;
+        // This warpgroup's column groups of the chunk: gg = w + 2u, u = 0..3.
+        // Pass 1: minimum of each group (two groups per TMEM wait, four
+        // independent min chains).  Columns past C_pad see cn = +inf; stale
+        // TMEM there turns into +inf or NaN, and NaN never wins a comparison.
+        float gmin[4];
+#pragma unroll
+        for (int u = 0; u < 4; u += 2) {
+          const int ga = w + 2 * u, gb = w + 2 * (u + 1);
+          uint32_t va[32], vb[32];
+          const bool has_a = ga * 32 < n, has_b = gb * 32 < n;
+          if (has_a) tmem_ld32(tbuf + 32 * ga, va);
+          if (has_b) tmem_ld32(tbuf + 32 * gb, vb);
+          tmem_ld_wait();
+          gmin[u] = inf;
+          gmin[u + 1] = inf;
+          if (has_a) gmin[u] = group_min(va, cn + j * kColChunk + 32 * ga);
+          if (has_b) gmin[u + 1] = group_min(vb, cn + j * kColChunk + 32 * gb);
+        }
+        run = fminf(run, fminf(fminf(gmin[0], gmin[1]), fminf(gmin[2], gmin[3])));
+        // Pass 2: only groups whose minimum lies within the margin of the
+        // running minimum can hold candidates (usually one group).
+        const float thr = run + margin;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int gg = w + 2 * u;
+          if (!__any_sync(0xffffffffu, gmin[u] <= thr)) continue;  // warp-uniform: tcgen05.ld
+          uint32_t v[32];
+          tmem_ld32(tbuf + 32 * gg, v);
+          tmem_ld_wait();
+          if (gmin[u] > thr) continue;
+          const int cbase = j * kColChunk + 32 * gg;
+          uint32_t hit = group_hits(v, cn + cbase, thr);
+          while (hit) {
+            const int k = __ffs(hit) - 1;
+            hit &= hit - 1;
+            uint32_t vk = 0;  // v[k] with a static index, so v stays in registers
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) vk = kk == k ? v[kk] : vk;
+            const float dv = fmaf(-2.f, __uint_as_float(vk), cn[cbase + k]);
+            c3 = c2; d3 = d2; c2 = c1; d2 = d1; c1 = c0; d1 = d0;
+            c0 = cbase + k; d0 = dv;
+            ++nc;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[kBarTmEmpty + b]);
+      }
+      const int xo = (t & 1) * kTileRows + r;
+      if (w == 1) {
+        xrun[xo] = run;
+        xcnt[xo] = nc;
+        xcand[4 * xo + 0] = c0; xcand[4 * xo + 1] = c1; xcand[4 * xo + 2] = c2; xcand[4 * xo + 3] = c3;
+        xdist[4 * xo + 0] = d0; xdist[4 * xo + 1] = d1; xdist[4 * xo + 2] = d2; xdist[4 * xo + 3] = d3;
+      }
+      named_bar(1, 256);
+      if (w == 0 && ok) {
+        const float best = fminf(run, xrun[xo]);
+        const float lim = best + margin;
+        const int nc1 = xcnt[xo];
+        int cs[8];
+        float ds[8];
+        cs[0] = c0; cs[1] = c1; cs[2] = c2; cs[3] = c3;
+        ds[0] = d0; ds[1] = d1; ds[2] = d2; ds[3] = d3;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          cs[4 + u] = xcand[4 * xo + u];
+          ds[4 + u] = xdist[4 * xo + u];
+        }
+        int keep = 0, kc[4] = {0, 0, 0, 0};
+        bool full = nc > 4 || nc1 > 4 || cbad || !(margin < inf);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const bool live = (u < 4 ? u < nc : (u - 4) < nc1) && ds[u] <= lim;
+          if (live) {
+            if (keep < 4) {
+              kc[0] = keep == 0 ? cs[u] : kc[0];
+              kc[1] = keep == 1 ? cs[u] : kc[1];
+              kc[2] = keep == 2 ? cs[u] : kc[2];
+              kc[3] = keep == 3 ? cs[u] : kc[3];
+            }
+            ++keep;
+          }
+        }
+        full = full || keep == 0 || keep > 4;
+        bool moved = false, pick = false;
+        int old = -1;
+        if (valid) {
+          old = p.first ? -1 : p.labels[g];
+          if (!full && keep == 1) {
+            p.labels[g] = kc[0];
+            moved = kc[0] != old;
+          } else {
+            pick = !full;
+          }
+        }
+        const unsigned long long pr = warp_append(p.refine_count, valid && full);
+        if (valid && full) p.refine_rows[pr] = g;
+        const unsigned long long pp = warp_append(p.pick_count, pick);
+        if (pick) {
+          Pick e;
+          e.row = g;
+          e.n = keep;
+          e.cand[0] = kc[0]; e.cand[1] = kc[1]; e.cand[2] = kc[2]; e.cand[3] = kc[3];
+          e.pad = 0;
+          p.picks[pp] = e;
+        }
+        const unsigned long long pm = warp_append(p.move_count, moved);
+        if (moved) p.moves[pm] = Move{g, old, kc[0]};
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort) latch(status, EAR_ERR_TIMEOUT);
+}
+
+// X -> fp16 copy and ||x|| (fp32, rounded up); +inf if the copy overflows.
+// (Below the fp16 normal range the copy rounds with absolute error <= 2^-25,
+// which the certification margin covers.)
+// A row is D/8 lanes of 8 values (16-byte loads and stores).
+template <int D>
+__global__ void km_xprep(const uint16_t* __restrict__ X, __half* __restrict__ Xh,
+                         float* __restrict__ xnorm, int64_t rows) {
+  constexpr int kLanes = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanes;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanes, part = lane % kLanes;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t g0 = warp * kRowsPerWarp; g0 < rows; g0 += nw * kRowsPerWarp) {
+    const int64_t g = g0 + sub;
+    float ss = 0.f;
+    bool exact = true;
+    if (g < rows) {
+      const uint4 raw = reinterpret_cast<const uint4*>(X + g * D)[part];
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t out[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float lo = __uint_as_float(w4[u] << 16), hi = __uint_as_float(w4[u] & 0xFFFF0000u);
+        const __half hl = __float2half_rn(lo), hh = __float2half_rn(hi);
+        exact &= fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;  // else the copy overflows
+        ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        out[u] = (uint32_t)__half_as_ushort(hl) | ((uint32_t)__half_as_ushort(hh) << 16);
+      }
+      reinterpret_cast<uint4*>(Xh + g * D)[part] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off >= 1; off >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      exact = __shfl_xor_sync(0xffffffffu, (int)exact, off) && exact;
+    }
+    if (part == 0 && g < rows)
+      xnorm[g] = exact ? sqrtf(ss) * (1.f + 1.0e-6f) : __int_as_float(0x7f800000);
+  }
+}
+
+// A centroid value beyond the fp16 range has no finite copy: the slice is
+// flagged (every row then takes the fp64 decision) and the copy is zeroed.
+__device__ __forceinline__ void prep_row(const float* __restrict__ c, __half* __restrict__ ch,
+                                         float* __restrict__ cnorm, float* __restrict__ cmax,
+                                         int* __restrict__ cbad, int D, bool real) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+  bool finite = true;
+  for (int k = lane; k < D; k += 32) {
+    const float v = real ? c[k] : 0.f;
+    finite &= fabsf(v) <= 65504.f;
+    ss = fmaf(v, v, ss);
+  }
+  finite = __all_sync(0xffffffffu, finite);
+  for (int k = lane; k < D; k += 32) ch[k] = __float2half_rn(finite && real ? c[k] : 0.f);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) {
+    *cnorm = real ? ss : __int_as_float(0x7f800000);
+    if (real) atomicMax(reinterpret_cast<int*>(cmax), __float_as_int(sqrtf(ss) * (1.f + 1.0e-6f)));
+    if (!finite) atomicOr(cbad, 1);
+  }
+}
+
+__global__ void km_cprep(const float* __restrict__ cent, __half* __restrict__ ch,
+                         float* __restrict__ cnorm, float* __restrict__ cmax,
+                         int* __restrict__ cbad, int C, int C_pad, int D, int64_t rows_pad) {
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= rows_pad) return;
+  const int64_t h = warp / C_pad;
+  const int c = (int)(warp % C_pad);
+  prep_row(cent + (h * C + (c < C ? c : 0)) * D, ch + warp * D, cnorm + warp, cmax + h, cbad + h,
+           D, c < C);
+}
+
+// exact fp64 argmin for the listed rows, then their moves
+template <typename T, int D>
+__global__ void km_refine64(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
+                            int C, int32_t* __restrict__ labels, int first,
+                            const int64_t* __restrict__ rows,
+                            const unsigned long long* __restrict__ count,
+                            float* __restrict__ sums, int32_t* __restrict__ cnt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = (int64_t)*count;
+  for (int64_t e = warp; e < total; e += nw) {
+    const int64_t g = rows[e];
+    const int64_t h = g / N;
+    const T* x = X + g * D;
+    const float* ch = cent + h * (int64_t)C * D;
+    double best = __longlong_as_double(0x7ff0000000000000ll);
+    int bidx = 0;
+    for (int c = lane; c < C; c += 32) {
+      const float* cc = ch + (int64_t)c * D;
+      double dist = 0.0;
+      for (int k = 0; k < D; ++k) {
+        const double diff = __dsub_rn((double)Elem<T>::load(x, k), (double)cc[k]);
+        dist = __dadd_rn(dist, __dmul_rn(diff, diff));
+      }
+      if (dist < best) {
+        best = dist;
+        bidx = c;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+      if (ob < best || (ob == best && oi < bidx)) {
+        best = ob;
+        bidx = oi;
+      }
+    }
+    const int old = first ? -1 : labels[g];
+    __syncwarp();
+    if (lane == 0) labels[g] = bidx;
+    if (bidx != old) {
+      for (int k = lane * 4; k < D; k += 128) {
+        const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
+                                     Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
+        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + bidx) * D + k), v);
+        if (old >= 0)
+          atomicAdd(reinterpret_cast<float4*>(sums + (h * C + old) * D + k),
+                    make_float4(-v.x, -v.y, -v.z, -v.w));
+      }
+      if (lane == 0) {
+        atomicAdd(cnt + h * C + bidx, 1);
+        if (old >= 0) atomicAdd(cnt + h * C + old, -1);
+      }
+    }
+  }
+}
+
+// fp64 decision among a row's 2-4 candidates (lane u takes candidate u),
+// then the move.
+template <typename T, int D>
+__global__ void km_pick64(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
+                          int C, int32_t* __restrict__ labels, int first,
+                          const Pick* __restrict__ picks,
+                          const unsigned long long* __restrict__ count,
+                          float* __restrict__ sums, int32_t* __restrict__ cnt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = (int64_t)*count;
+  for (int64_t e = warp; e < total; e += nw) {
+    const Pick pk = picks[e];
+    const int64_t g = pk.row;
+    const int64_t h = g / N;
+    const T* x = X + g * D;
+    double best = __longlong_as_double(0x7ff0000000000000ll);
+    int bidx = C;
+    if (lane < pk.n) {
+      const int c = pk.cand[lane];
+      const float* cc = cent + (h * C + c) * (int64_t)D;
+      double dist = 0.0;
+      for (int k = 0; k < D; ++k) {
+        const double diff = __dsub_rn((double)Elem<T>::load(x, k), (double)cc[k]);
+        dist = __dadd_rn(dist, __dmul_rn(diff, diff));
+      }
+      best = dist;
+      bidx = c;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+      if (ob < best || (ob == best && oi < bidx)) {
+        best = ob;
+        bidx = oi;
+      }
+    }
+    const int old = first ? -1 : labels[g];
+    __syncwarp();
+    if (lane == 0) labels[g] = bidx;
+    if (bidx != old) {
+      for (int k = lane * 4; k < D; k += 128) {
+        const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
+                                     Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
+        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + bidx) * D + k), v);
+        if (old >= 0)
+          atomicAdd(reinterpret_cast<float4*>(sums + (h * C + old) * D + k),
+                    make_float4(-v.x, -v.y, -v.z, -v.w));
+      }
+      if (lane == 0) {
+        atomicAdd(cnt + h * C + bidx, 1);
+        if (old >= 0) atomicAdd(cnt + h * C + old, -1);
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void km_moves(const T* __restrict__ X, int64_t N, int C, const Move* __restrict__ moves,
+                         const unsigned long long* __restrict__ count, float* __restrict__ sums,
+                         int32_t* __restrict__ cnt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = (int64_t)*count;
+  for (int64_t e = warp; e < total; e += nw) {
+    const Move mv = moves[e];
+    const int64_t h = mv.row / N;
+    const T* x = X + mv.row * D;
+    for (int k = lane * 4; k < D; k += 128) {
+      const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
+                                   Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
+      atomicAdd(reinterpret_cast<float4*>(sums + (h * C + mv.to) * D + k), v);
+      if (mv.from >= 0)
+        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + mv.from) * D + k),
+                  make_float4(-v.x, -v.y, -v.z, -v.w));
+    }
+    if (lane == 0) {
+      atomicAdd(cnt + h * C + mv.to, 1);
+      if (mv.from >= 0) atomicAdd(cnt + h * C + mv.from, -1);
+    }
+  }
+}
+
+// new centroids from the running sums, then the fp16 / norm copies
+__global__ void km_finalize(const float* __restrict__ sums, const int32_t* __restrict__ cnt,
+                            float* __restrict__ cent, int32_t* __restrict__ counts,
+                            __half* __restrict__ ch, float* __restrict__ cnorm,
+                            float* __restrict__ cmax, int* __restrict__ cbad, int C, int C_pad,
+                            int D, int64_t rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= rows) return;  // rows = BH * C
+  const int64_t h = warp / C;
+  const int c = (int)(warp % C);
+  const int n = cnt[warp];
+  float* cr = cent + warp * D;
+  if (n > 0)
+    for (int k = lane; k < D; k += 32) cr[k] = sums[warp * D + k] / (float)n;
+  if (lane == 0) counts[warp] = n;
+  __syncwarp();
+  prep_row(cr, ch + (h * C_pad + c) * D, cnorm + h * C_pad + c, cmax + h, cbad + h, D, true);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+bool make_map_f16(CUtensorMap* map, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcWs {
+  float* sums;
+  int32_t* cnt;
+  int64_t* refine_rows;
+  unsigned long long* counters;  // [0] full refine, [1] moves, [2] picks
+  Pick* picks;
+  Move* moves;
+  __half* xh;
+  float* xnorm;
+  __half* ch;
+  float* cnorm;
+  float* cmax;  // [BH] floats, then [BH] ints (cbad): cleared together
+  int* cbad;
+};
+
+int c_pad_of(int32_t c) { return (int)ceil_div(c, 16) * 16; }
+
+TcWs carve(Carver& cv, int64_t bh, int64_t n, int32_t d, int32_t c) {
+  TcWs w;
+  const int cp = c_pad_of(c);
+  w.sums = cv.take<float>((size_t)bh * c * d);
+  w.cnt = cv.take<int32_t>((size_t)bh * c);
+  w.refine_rows = cv.take<int64_t>((size_t)bh * n);
+  w.counters = cv.take<unsigned long long>(3);
+  w.picks = cv.take<Pick>((size_t)bh * n);
+  w.moves = cv.take<Move>((size_t)bh * n);
+  w.xh = cv.take<__half>((size_t)bh * n * d);
+  w.xnorm = cv.take<float>((size_t)bh * n);
+  w.ch = cv.take<__half>((size_t)bh * cp * d);
+  w.cnorm = cv.take<float>((size_t)bh * cp);
+  w.cmax = cv.take<float>((size_t)bh * 2);
+  w.cbad = reinterpret_cast<int*>(w.cmax + bh);
+  return w;
+}
+
+template <int D>
+ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t iters,
+                  const float* init, float* cent, int32_t* labels, int32_t* counts, void* ws,
+                  cudaStream_t s) {
+  using L = KLayout<D>;
+  Carver cv(ws);
+  TcWs w = carve(cv, bh, n, D, c);
+  const int cp = c_pad_of(c);
+  int* status = device_status_word();
+  const int64_t rows = bh * n;
+  const unsigned wgrid = (unsigned)std::min<int64_t>(ceil_div(rows, 8), 148 * 32);
+
+  if (cent != init)
+    EAR_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * bh * c * D, cudaMemcpyDeviceToDevice, s));
+  EAR_CUDA(cudaMemsetAsync(w.sums, 0, sizeof(float) * bh * c * D, s));
+  EAR_CUDA(cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * bh * c, s));
+  km_xprep<D><<<wgrid, 256, 0, s>>>(X, w.xh, w.xnorm, rows);
+  EAR_TRY(after_launch());
+  EAR_CUDA(cudaMemsetAsync(w.cmax, 0, sizeof(float) * bh * 2, s));
+  const int64_t prow = bh * cp;
+  km_cprep<<<(unsigned)ceil_div(prow, 8), 256, 0, s>>>(cent, w.ch, w.cnorm, w.cmax, w.cbad, c, cp,
+                                                        D, prow);
+  EAR_TRY(after_launch());
+
+  CUtensorMap mx, mc;
+  const int c_box = std::min(cp, kColChunk);
+  if (!make_map_f16(&mx, w.xh, rows, D, kTileRows) || !make_map_f16(&mc, w.ch, bh * cp, D, c_box))
+    return EAR_ERR_CUDA;
+  KmTcParams p;
+  p.xnorm = w.xnorm;
+  p.cnorm = w.cnorm;
+  p.cmax = w.cmax;
+  p.cbad = w.cbad;
+  p.labels = labels;
+  p.refine_rows = w.refine_rows;
+  p.refine_count = w.counters;
+  p.moves = w.moves;
+  p.move_count = w.counters + 1;
+  p.picks = w.picks;
+  p.pick_count = w.counters + 2;
+  p.N = n;
+  p.C = c;
+  p.C_pad = cp;
+  p.c_box = c_box;
+  const double a = 2.0 * (std::ldexp(1.0, -11) + (D + 1) * std::ldexp(1.0, -23)) *
+                   (1.0 + std::ldexp(1.0, -11)) * (1.0 + std::ldexp(1.0, -20));
+  p.a_coef = (float)(a * (1.0 + 1e-6));
+  p.b_coef = (float)std::ldexp(1.0, -16);
+  // centroid values in the fp16 subnormal range round with absolute error
+  // <= 2^-25: at most sqrt(d) 2^-25 ||x|| on x.c, doubled in d~
+  p.s_coef = (float)(2.0 * std::sqrt((double)D) * std::ldexp(1.0, -25) * 1.01);
+  EAR_CUDA(cudaFuncSetAttribute(km_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  const dim3 grid((unsigned)ceil_div(ceil_div(n, kTileRows), kTilesPerCta), (unsigned)bh);
+  const int64_t crow = bh * (int64_t)c;
+  for (int t = 0; t < iters; ++t) {
+    p.first = t == 0 ? 1 : 0;
+    EAR_CUDA(cudaMemsetAsync(w.counters, 0, 3 * sizeof(unsigned long long), s));
+    km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
+    EAR_TRY(after_launch());
+    km_refine64<uint16_t, D><<<wgrid, 256, 0, s>>>(X, cent, n, c, labels, p.first, w.refine_rows,
+                                                   w.counters, w.sums, w.cnt);
+    EAR_TRY(after_launch());
+    km_pick64<uint16_t, D><<<wgrid, 256, 0, s>>>(X, cent, n, c, labels, p.first, w.picks,
+                                                 w.counters + 2, w.sums, w.cnt);
+    EAR_TRY(after_launch());
+    km_moves<uint16_t, D><<<wgrid, 256, 0, s>>>(X, n, c, w.moves, w.counters + 1, w.sums, w.cnt);
+    EAR_TRY(after_launch());
+    EAR_CUDA(cudaMemsetAsync(w.cmax, 0, sizeof(float) * bh * 2, s));
+    km_finalize<<<(unsigned)ceil_div(crow, 8), 256, 0, s>>>(w.sums, w.cnt, cent, counts, w.ch,
+                                                           w.cnorm, w.cmax, w.cbad, c, cp, D,
+                                                           crow);
+    EAR_TRY(after_launch());
+  }
+  return EAR_OK;
+}
+
+}  // namespace
+
+bool kmeans_tc_supported(ear_dtype dt, int32_t d, int32_t c) {
+  return dt == EAR_BF16 && (d == 64 || d == 128) && c_pad_of(c) <= kMaxCPad;
+}
+
+size_t kmeans_tc_workspace(int64_t bh, int64_t n, int32_t d, int32_t c) {
+  Carver cv(nullptr);
+  carve(cv, bh, n, d, c);
+  return cv.used;
+}
+
+ear_status kmeans_tc_run(const void* X, int64_t bh, int64_t n, int32_t d, int32_t c,
+                         int32_t iters, const float* init, float* cent, int32_t* labels,
+                         int32_t* counts, void* ws, cudaStream_t s) {
+  const uint16_t* x = static_cast<const uint16_t*>(X);
+  return d == 64 ? run_tc<64>(x, bh, n, c, iters, init, cent, labels, counts, ws, s)
+                 : run_tc<128>(x, bh, n, c, iters, init, cent, labels, counts, ws, s);
+}
+
+}  // namespace ear

@@ -78,6 +78,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait whose result is the same in every lane of the warp (needed
+// before .sync.aligned instructions such as tcgen05.ld).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Teardown wait: ignores the abort flag (the work it waits for is already in
 // flight and must land before the CTA exits) but still gives up after kWaitNs.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {

@@ -93,6 +93,49 @@ def test_kmeans_all_iterations(layers, cfg):
             np.testing.assert_allclose(cent[h], c_ref, rtol=0, atol=1e-5 * np.abs(c_ref).max())
 
 
+@pytest.mark.parametrize("n,c,d,iters", [(3001, 500, 64, 4), (2000, 300, 128, 3),
+                                         (777, 17, 128, 5), (4096, 512, 128, 2)])
+def test_kmeans_tensor_core_path_shapes(n, c, d, iters):
+    """bf16 k-means with C <= 512 runs on the tensor cores: two 256-column
+    chunks, a partial last column group, ragged row tiles."""
+    w = gen.MID.with_(heads=2, n=n, d=d, n_centres=max(c // 3, 4), c_q=c, c_k=c, iters=iters)
+    L = gen.make_layer(w)
+    for it in (1, iters):
+        cent, lab, cnt = ear.ear_kmeans(pu.dev(L.k, torch.bfloat16), pu.dev(L.k_init), it)
+        cent, lab, cnt = pu.host(cent), pu.host(lab), pu.host(cnt)
+        for h in range(2):
+            c_ref, l_ref, n_ref = eo.kmeans(L.k[h], L.k_init[h], it)
+            prev = L.k_init[h] if it == 1 else eo.kmeans(L.k[h], L.k_init[h], it - 1)[0]
+            bad = np.nonzero(lab[h] != l_ref)[0]
+            for i in bad:  # only near-ties under the centroids the last assignment used
+                x = L.k[h][i].astype(np.float64)
+                dg = ((x - prev[lab[h][i]]) ** 2).sum()
+                dr = ((x - prev[l_ref[i]]) ** 2).sum()
+                tol = pu.TIE_REL if it == 1 else 1e-4
+                assert abs(dg - dr) <= tol * ((x ** 2).sum() + (prev[l_ref[i]] ** 2).sum())
+            assert cnt[h].sum() == n
+            np.testing.assert_array_equal(cnt[h], np.bincount(lab[h], minlength=c))
+            if len(bad) == 0:
+                np.testing.assert_allclose(cent[h], c_ref, rtol=0, atol=1e-5 * np.abs(c_ref).max())
+
+
+def test_kmeans_rows_outside_fp16_are_decided_exactly():
+    """Values with no exact fp16 copy (above 65504, or too small) send their
+    rows through the fp64 decision; labels still match the oracle."""
+    rng = np.random.default_rng(3)
+    n, c, d = 1500, 40, 128
+    x = rng.standard_normal((1, n, d))
+    x[0, 10, 5] = 1.0e5
+    x[0, 11, :] = 3.0e-8
+    x[0, 12, 7] = -7.0e4
+    x = gen.round_to_bf16(x)
+    init = np.ascontiguousarray(x[:, rng.choice(n, c, replace=False)])
+    init[0, 0] = x[0, 10]
+    _, lab, _ = ear.ear_kmeans(pu.dev(x, torch.bfloat16), pu.dev(init), 1)
+    _, l_ref, _ = eo.kmeans(x[0], init[0], 1)
+    pu.assert_labels_exact_or_tie(x[0], init[0], pu.host(lab)[0], l_ref)
+
+
 # --------------------------------------------------------------------------- permutation
 @pytest.mark.parametrize("n,c,dtype,d", [(8192, 128, "bf16", 128), (1000, 7, "f32", 64),
                                          (3001, 40, "bf16", 64), (5, 3, "f32", 128)])
