@@ -4,23 +4,29 @@
 //
 // One CTA = one unit of up to 256 permuted query rows of ONE query cluster a,
 // split in two 128-row tiles A and B (tcgen05.mma M = 128).  Both tiles walk
-// the same key chunks:
-//   * exact chunks: every key cluster b listed for a, in pieces of <= 128
-//     keys taken straight from the permuted K / V rows;
-//   * compensation chunks (EAR_COMPENSATE): the C_k key / value centroids in
-//     pieces of 128, with per-column bias log2|b| (weight |b|) and -inf for
-//     clusters that are exact for a or empty.
+// the same key chunks.  A chunk is up to four 32-row boxes (128 keys):
+//   * exact boxes: the rows of every key cluster b listed for a, 32 at a
+//     time (the last box of a cluster is partial), so small clusters share
+//     a chunk instead of each paying for a whole MMA round;
+//   * compensation boxes (EAR_COMPENSATE): the C_k key / value centroids, 32
+//     at a time, with per-column bias log2|b| (weight |b|) and -inf for
+//     clusters that are exact for a or empty.  Exact and centroid boxes never
+//     share a chunk.
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then K/V chunks into a 2-stage ring;
-//               computes the compensation bias of each centroid chunk.
+//   warp 0      TMA producer: Q tiles once, then chunk boxes into a 2-stage
+//               ring.  It publishes each stage's chunk descriptor (box count,
+//               valid rows per box, centroid or not, bias) in shared memory
+//               and ends the sequence with an empty descriptor.
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T into TMEM, then
 //               O_t += P_t V with P_t read from TMEM.  Issue order
 //               QK_A(c) QK_B(c) | PV_A(c) QK_A(c+1) PV_B(c) QK_B(c+1) | ...
 //               so one tile's softmax overlaps the other tile's MMAs.
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread
-//               per query row (= TMEM lane).  Online softmax in base 2; the
-//               running max is only moved (and O rescaled in TMEM) when it
-//               grows by more than 2^8, so most chunks skip the rescale.
+//               per query row (= TMEM lane).  Online softmax in base 2 on the
+//               raw scores: the max pass is one compare per score, the
+//               exponent argument one packed FMA per score pair; the running
+//               max only moves (and O is rescaled in TMEM) when it grows by
+//               more than 2^8.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512);
 // P_t (bf16 pairs) overwrites the first half of S_t.
 #include <mutex>
@@ -36,9 +42,10 @@ using namespace sm100;
 constexpr int kTileRows = 128;
 constexpr int kTiles = 2;
 constexpr int kUnitRows = kTileRows * kTiles;
-constexpr int kChunk = 128;
+constexpr int kBox = 32;                 // rows per TMA box
+constexpr int kBoxes = 4;                // boxes per chunk
+constexpr int kChunk = kBox * kBoxes;    // keys per chunk (MMA N <= 128)
 constexpr int kStages = 2;
-constexpr int kBoxRows = 32;
 constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -54,6 +61,13 @@ constexpr int kBarODone = 9;    // + tile
 constexpr int kBarDrain = 11;   // teardown: every MMA issued has finished
 constexpr int kNumBars = 12;
 
+// Chunk descriptor published by the producer for each stage.
+struct ChunkInfo {
+  int32_t nbox;          // 0 = no more chunks
+  int32_t comp;          // centroid chunk
+  int32_t valid[kBoxes]; // valid rows of each box (1..32)
+};
+
 template <int D>
 struct Layout {
   static constexpr int kHalfBytes = kTileRows * 128;  // 128 rows x 64 bf16
@@ -61,8 +75,9 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTiles * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBias = kV + kStages * kTileBytes;
-  static constexpr int kBar = kBias + kStages * kChunk * 4;
+  static constexpr int kBias = kV + kStages * kTileBytes;       // [stage][128] float
+  static constexpr int kInfo = kBias + kStages * kChunk * 4;    // [stage] ChunkInfo
+  static constexpr int kBar = kInfo + kStages * 32;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -86,8 +101,9 @@ struct TcParams {
   int* status;
 };
 
-// The chunk sequence of one unit; every role walks its own copy.
-struct Chunks {
+// Box sequence of one unit (producer only): the rows of each exact key
+// cluster in 32-row boxes, then the centroids in 32-row boxes.
+struct Boxes {
   const int32_t* list;
   const int32_t* koff;
   int32_t e, e1, pos, end;
@@ -108,9 +124,9 @@ struct Chunks {
     compensate = p.compensate;
     status = p.status;
   }
-  // row: first key row within the slice (exact) or first centroid (compensation);
-  // comp = whether this is a centroid chunk.
-  __device__ bool next(int32_t& row, int& nv, bool& comp) {
+  // Next box: first row (key row in the slice, or centroid index), valid
+  // rows, and whether it is a centroid box.  False when none is left.
+  __device__ bool next(int32_t& row, int& valid, bool& comp) {
     while (pos >= end && e < e1) {
       const int b = list[e++];
       if (b < 0 || b >= Ck) {
@@ -126,15 +142,15 @@ struct Chunks {
     }
     if (pos < end) {
       row = pos;
-      nv = min(kChunk, end - pos);
-      pos += nv;
+      valid = min(kBox, end - pos);
+      pos += valid;
       comp = false;
       return true;
     }
     if (compensate && comp_next < Ck) {
       row = comp_next;
-      nv = min(kChunk, Ck - comp_next);
-      comp_next += kChunk;
+      valid = min(kBox, Ck - comp_next);
+      comp_next += kBox;
       comp = true;
       return true;
     }
@@ -142,7 +158,71 @@ struct Chunks {
   }
 };
 
-__device__ __forceinline__ int round_up(int x, int m) { return (x + m - 1) / m * m; }
+__device__ __forceinline__ unsigned long long pack2(uint32_t lo, uint32_t hi) {
+  return (unsigned long long)lo | ((unsigned long long)hi << 32);
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float lo_f(unsigned long long x) { return __uint_as_float((uint32_t)x); }
+__device__ __forceinline__ float hi_f(unsigned long long x) {
+  return __uint_as_float((uint32_t)(x >> 32));
+}
+
+// max of 32 raw scores, columns >= valid excluded
+__device__ __forceinline__ float box_max_raw(const uint32_t (&v)[32], int valid) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  if (valid >= 32) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m[j & 3] = fmaxf(m[j & 3], __uint_as_float(v[j]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      m[j & 3] = fmaxf(m[j & 3], j < valid ? __uint_as_float(v[j]) : -INFINITY);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// max of 32 scaled-and-biased scores (centroid box)
+__device__ __forceinline__ float box_max_bias(const uint32_t (&v)[32], const float* bias,
+                                              float scale, int valid) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float z = fmaf(__uint_as_float(v[j]), scale, bias[j]);
+    m[j & 3] = fmaxf(m[j & 3], j < valid ? z : -INFINITY);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p = 2^(score * scale + shift_j) for 32 columns (shift pairs from `sh`),
+// packed to bf16 pairs; returns the two partial row sums as a pair.
+__device__ __forceinline__ unsigned long long box_exp(const uint32_t (&v)[32],
+                                                      const unsigned long long (&sh)[16],
+                                                      unsigned long long scale2, int valid,
+                                                      uint32_t (&pk)[16]) {
+  unsigned long long sum = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const unsigned long long z = fma2(pack2(v[j], v[j + 1]), scale2, sh[j / 2]);
+    float p0 = ex2(lo_f(z)), p1 = ex2(hi_f(z));
+    if (valid < 32) {
+      p0 = j < valid ? p0 : 0.f;
+      p1 = j + 1 < valid ? p1 : 0.f;
+    }
+    sum = add2(sum, pack2(__float_as_uint(p0), __float_as_uint(p1)));
+    pk[j / 2] = pack_bf16x2(p0, p1);
+  }
+  return sum;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -165,13 +245,15 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
     if (threadIdx.x == 0) latch(p.status, EAR_ERR_DEVICE);
     return;
   }
-  const int rows_t[2] = {min(kTileRows, qend - row0), max(0, min(kTileRows, qend - row0 - kTileRows))};
-  const int ntiles = rows_t[1] > 0 ? 2 : 1;
+  const int rows_a = min(kTileRows, qend - row0);
+  const int rows_b = max(0, min(kTileRows, qend - row0 - kTileRows));
+  const int ntiles = rows_b > 0 ? 2 : 1;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   float* bias = reinterpret_cast<float*>(smem + L::kBias);
+  ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -212,22 +294,36 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
           tma_load_2d(smem + L::kQ + t * L::kTileBytes + hf * L::kHalfBytes, &tmQ,
                       &bars[kBarQFull], 64 * hf, (int32_t)(h * p.Nq) + row0 + kTileRows * t);
     }
-    Chunks it;
+    Boxes it;
     it.init(p, h, a);
-    int32_t row;
-    int nv;
-    bool comp;
+    int32_t brow = 0;
+    int bval = 0;
+    bool bcomp = false;
+    bool have = it.next(brow, bval, bcomp);  // the box that opens the next chunk
     int issued = 0;
-    for (int c = 0; it.next(row, nv, comp); ++c) {
+    for (int c = 0;; ++c) {
       const int s = c % kStages;
       if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
         break;
       issued = c + 1;
-      if (comp) {
+      ChunkInfo ci;
+      ci.nbox = 0;
+      ci.comp = have && bcomp ? 1 : 0;
+      int32_t rows[kBoxes];
+      const int32_t comp_first = brow;
+      // up to four boxes of the same kind
+      while (have && ci.nbox < kBoxes && (bcomp ? 1 : 0) == ci.comp) {
+        rows[ci.nbox] = brow;
+        ci.valid[ci.nbox] = bval;
+        ++ci.nbox;
+        have = it.next(brow, bval, bcomp);
+      }
+      if (ci.comp) {  // bias of the chunk's columns (centroids comp_first ...)
         for (int j = lane; j < kChunk; j += 32) {
           float bv = -INFINITY;
-          if (j < nv) {
-            const int b = row + j;
+          const int bx = j / kBox;
+          if (bx < ci.nbox && (j % kBox) < ci.valid[bx]) {
+            const int b = comp_first + j;
             const int32_t cnt = koff[b + 1] - koff[b];
             if (!exact_row[b] && cnt > 0) bv = __log2f((float)cnt);
           }
@@ -236,26 +332,29 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
       }
       __syncwarp();
       if (lane == 0) {
-        const int npad = round_up(nv, kBoxRows);
-        mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * npad * D * 2);
-        const CUtensorMap* mk = comp ? &tmKc : &tmK;
-        const CUtensorMap* mv = comp ? &tmVc : &tmV;
-        const int32_t grow = comp ? (int32_t)(h * p.Ck_pad) + row : (int32_t)(h * p.Nk) + row;
-        uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
-        uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
-        for (int r = 0; r < npad; r += kBoxRows)
-          for (int hf = 0; hf < D / 64; ++hf) {
-            tma_load_2d(kdst + hf * L::kHalfBytes + r * 128, mk, &bars[kBarKvFull + s], 64 * hf,
-                        grow + r);
-            tma_load_2d(vdst + hf * L::kHalfBytes + r * 128, mv, &bars[kBarKvFull + s], 64 * hf,
-                        grow + r);
-          }
+        info[s] = ci;
+        if (ci.nbox == 0) {
+          mbar_arrive(&bars[kBarKvFull + s]);  // end of the sequence
+        } else {
+          mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * ci.nbox * kBox * D * 2);
+          const CUtensorMap* mk = ci.comp ? &tmKc : &tmK;
+          const CUtensorMap* mv = ci.comp ? &tmVc : &tmV;
+          const int32_t base = ci.comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
+          uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
+          uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
+          for (int bx = 0; bx < ci.nbox; ++bx)
+            for (int hf = 0; hf < D / 64; ++hf) {
+              tma_load_2d(kdst + hf * L::kHalfBytes + bx * kBox * 128, mk, &bars[kBarKvFull + s],
+                          64 * hf, base + rows[bx]);
+              tma_load_2d(vdst + hf * L::kHalfBytes + bx * kBox * 128, mv, &bars[kBarKvFull + s],
+                          64 * hf, base + rows[bx]);
+            }
+        }
       }
       __syncwarp();
+      if (ci.nbox == 0) break;
     }
-    // Teardown after an abort: let the loads already issued land before the
-    // CTA exits (a no-op when the consumers saw every chunk).
-    if (*abort) {
+    if (*abort) {  // let issued loads land before the CTA exits
       mbar_wait_drain(&bars[kBarQFull], 0);
       for (int c = issued - 1; c >= 0 && c >= issued - kStages; --c)
         mbar_wait_drain(&bars[kBarKvFull + c % kStages], (c / kStages) & 1);
@@ -282,32 +381,19 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
                  desc_sw128(vb + kk * 2048, L::kHalfBytes, 1024), idesc_pv,
                  (first && kk == 0) ? 0u : 1u);
       };
-      Chunks it;
-      it.init(p, h, a);
-      int32_t row;
-      int nv;
-      bool comp;
-      bool have = it.next(row, nv, comp);
-      int n_cur = round_up(nv, 16);
-      bool ok = mbar_wait(&bars[kBarQFull], 0, abort);
-      if (ok && have) {
-        ok = mbar_wait(&bars[kBarKvFull + 0], 0, abort);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < ntiles; ++t) {
-            issue_qk(t, 0, n_cur);
-            mma_commit(&bars[kBarSFull + t]);
-          }
+      bool ok = mbar_wait(&bars[kBarQFull], 0, abort) && mbar_wait(&bars[kBarKvFull], 0, abort);
+      int n_cur = ok ? info[0].nbox * kBox : 0;
+      if (ok && n_cur > 0) {
+        tc_fence_after();
+        for (int t = 0; t < ntiles; ++t) {
+          issue_qk(t, 0, n_cur);
+          mma_commit(&bars[kBarSFull + t]);
         }
       }
-      for (int c = 0; ok && have; ++c) {
+      for (int c = 0; ok && n_cur > 0; ++c) {
         const int s = c % kStages;
         const int s2 = (c + 1) % kStages;
-        int32_t row2;
-        int nv2;
-        bool comp2;
-        const bool have2 = it.next(row2, nv2, comp2);
-        const int n_nxt = round_up(nv2, 16);
+        int n_nxt = 0;
         for (int t = 0; t < ntiles && ok; ++t) {
           ok = mbar_wait(&bars[kBarPFull + t], c & 1, abort);
           if (!ok) break;
@@ -315,17 +401,17 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
           issue_pv(t, s, n_cur, c == 0);
           mma_commit(&bars[kBarODone + t]);
           if (t == ntiles - 1) mma_commit(&bars[kBarKvEmpty + s]);
-          if (have2) {
-            if (t == 0) {
-              ok = mbar_wait(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
-              if (!ok) break;
-              tc_fence_after();
-            }
+          if (t == 0) {
+            ok = mbar_wait(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
+            if (!ok) break;
+            n_nxt = info[s2].nbox * kBox;
+            tc_fence_after();
+          }
+          if (n_nxt > 0) {
             issue_qk(t, s2, n_nxt);
             mma_commit(&bars[kBarSFull + t]);
           }
         }
-        have = have2;
         n_cur = n_nxt;
       }
       // every MMA issued above has finished before TMEM is released
@@ -337,37 +423,44 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
     const int t = (warp - 4) / 4;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row within the tile = TMEM lane
+    const int rows_t = t == 0 ? rows_a : rows_b;
     if (t < ntiles) {
       const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
       const uint32_t tS = tmem + lane_bits + kTileRows * t;
       const uint32_t tO = tmem + lane_bits + 256 + kTileRows * t;
-      float m = -INFINITY, l = 0.f;
-      Chunks it;
-      it.init(p, h, a);
-      int32_t row;
-      int nv;
-      bool comp;
+      const float scale = p.qk_scale;
+      const unsigned long long scale2 = pack2(__float_as_uint(scale), __float_as_uint(scale));
+      float m = -INFINITY;                  // running max (scaled, base 2)
+      unsigned long long lsum = 0;          // running sum as two partial sums
       int c = 0;
       bool ok = true;
-      uint32_t v[32];
-      for (; it.next(row, nv, comp); ++c) {
+      for (;; ++c) {
         const int s = c % kStages;
+        ok = mbar_wait_warp(&bars[kBarKvFull + s], (c / kStages) & 1, abort);
+        if (!ok) break;
+        const ChunkInfo* ci = &info[s];  // read in place (runtime box index)
+        const int nbox = ci->nbox;
+        const bool comp = ci->comp != 0;
+        if (nbox == 0) break;
         ok = mbar_wait_warp(&bars[kBarSFull + t], c & 1, abort);
-        if (ok && comp) ok = mbar_wait_warp(&bars[kBarKvFull + s], (c / kStages) & 1, abort);
         if (!ok) break;
         tc_fence_after();
         const float* bs = bias + s * kChunk;
-        const int ng = (nv + 31) / 32;
+        // pass 1: chunk max (scaled)
         float mx = -INFINITY;
-        for (int g = 0; g < ng; ++g) {
-          tmem_ld32(tS + 32 * g, v);
+        for (int bx = 0; bx < nbox; bx += 2) {
+          uint32_t va[32], vb[32];
+          const bool has_b = bx + 1 < nbox;
+          tmem_ld32(tS + 32 * bx, va);
+          if (has_b) tmem_ld32(tS + 32 * (bx + 1), vb);
           tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = 32 * g + j;
-            float z = __uint_as_float(v[j]) * p.qk_scale + (comp ? bs[col] : 0.f);
-            z = col < nv ? z : -INFINITY;
-            mx = fmaxf(mx, z);
+          const int v0 = ci->valid[bx], v1 = has_b ? ci->valid[bx + 1] : 0;
+          if (!comp) {
+            mx = fmaxf(mx, box_max_raw(va, v0) * scale);
+            if (has_b) mx = fmaxf(mx, box_max_raw(vb, v1) * scale);
+          } else {
+            mx = fmaxf(mx, box_max_bias(va, bs + 32 * bx, scale, v0));
+            if (has_b) mx = fmaxf(mx, box_max_bias(vb, bs + 32 * (bx + 1), scale, v1));
           }
         }
         float m_use = m, corr = 1.f;
@@ -379,22 +472,28 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
           }
           m_use = mx;
         }
-        l *= corr;
-        for (int g = 0; g < ng; ++g) {
-          tmem_ld32(tS + 32 * g, v);
+        if (resc) lsum = pack2(__float_as_uint(lo_f(lsum) * corr), __float_as_uint(hi_f(lsum) * corr));
+        // pass 2: P = 2^(scaled score - m_use) into the first half of S
+        const float neg = m_use == -INFINITY ? 0.f : -m_use;  // all scores -inf: p = 0 below
+        for (int bx = 0; bx < nbox; ++bx) {
+          uint32_t v[32];
+          tmem_ld32(tS + 32 * bx, v);
           tmem_ld_wait();
-          uint32_t pk[16];
+          unsigned long long sh[16];
+          if (!comp) {
+            const unsigned long long n2 = pack2(__float_as_uint(neg), __float_as_uint(neg));
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int col = 32 * g + j;
-            float z0 = __uint_as_float(v[j]) * p.qk_scale + (comp ? bs[col] : 0.f);
-            float z1 = __uint_as_float(v[j + 1]) * p.qk_scale + (comp ? bs[col + 1] : 0.f);
-            const float p0 = (col < nv && m_use != -INFINITY) ? ex2(z0 - m_use) : 0.f;
-            const float p1 = (col + 1 < nv && m_use != -INFINITY) ? ex2(z1 - m_use) : 0.f;
-            l += p0 + p1;
-            pk[j / 2] = pack_bf16x2(p0, p1);
+            for (int j = 0; j < 16; ++j) sh[j] = n2;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              sh[j] = pack2(__float_as_uint(bs[32 * bx + 2 * j] + neg),
+                            __float_as_uint(bs[32 * bx + 2 * j + 1] + neg));
           }
-          tmem_st16(tS + 16 * g, pk);
+          const int valid = m_use == -INFINITY ? 0 : ci->valid[bx];
+          uint32_t pk[16];
+          lsum = add2(lsum, box_exp(v, sh, scale2, valid, pk));
+          tmem_st16(tS + 16 * bx, pk);
         }
         tmem_st_wait();
         if (__any_sync(0xffffffffu, resc)) {
@@ -402,6 +501,7 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
           if (!ok) break;
           tc_fence_after();
           for (int g = 0; g < D / 32; ++g) {
+            uint32_t v[32];
             tmem_ld32(tO + 32 * g, v);
             tmem_ld_wait();
 #pragma unroll
@@ -415,15 +515,17 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
         mbar_arrive(&bars[kBarPFull + t]);
       }
       // epilogue: O / l written at the queries' original positions
+      const float l = lo_f(lsum) + hi_f(lsum);
       const int32_t prow = row0 + kTileRows * t + r;
-      const int32_t orig = r < rows_t[t] ? p.q_perm[h * p.Nq + prow] : -1;
+      const int32_t orig = r < rows_t ? p.q_perm[h * p.Nq + prow] : -1;
       const bool valid = orig >= 0 && orig < p.Nq;
-      if (r < rows_t[t] && !valid) latch(p.status, EAR_ERR_DEVICE);
+      if (r < rows_t && !valid) latch(p.status, EAR_ERR_DEVICE);
       const bool have_o = ok && c > 0 && mbar_wait_warp(&bars[kBarODone + t], (c - 1) & 1, abort);
       if (have_o) tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint16_t* orow = p.O + ((int64_t)h * p.Nq + (valid ? orig : 0)) * D;
       for (int g = 0; g < D / 32; ++g) {
+        uint32_t v[32];
         if (have_o) {
           tmem_ld32(tO + 32 * g, v);
           tmem_ld_wait();
@@ -512,10 +614,9 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
   EAR_TRY(after_launch());
   CUtensorMap mq, mk, mv, mkc, mvc;
   if (!make_map(&mq, a.Q, a.bh * a.n_q, D, kTileRows) ||
-      !make_map(&mk, a.K, a.bh * a.n_k, D, kBoxRows) ||
-      !make_map(&mv, a.V, a.bh * a.n_k, D, kBoxRows) ||
-      !make_map(&mkc, kc16, a.bh * ck_pad, D, kBoxRows) ||
-      !make_map(&mvc, vc16, a.bh * ck_pad, D, kBoxRows))
+      !make_map(&mk, a.K, a.bh * a.n_k, D, kBox) || !make_map(&mv, a.V, a.bh * a.n_k, D, kBox) ||
+      !make_map(&mkc, kc16, a.bh * ck_pad, D, kBox) ||
+      !make_map(&mvc, vc16, a.bh * ck_pad, D, kBox))
     return EAR_ERR_CUDA;
   TcParams p;
   p.q_off = a.q_off;

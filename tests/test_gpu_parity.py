@@ -271,7 +271,24 @@ def test_attention_given_same_mask(layers, oracle_runs, cfg, compensate):
         ok = np.isfinite(lse_ref)
         pu.assert_attention_close(o[h][ok], o_ref[ok], w.dtype)
         assert np.all(o[h][~ok] == 0) and np.all(np.isneginf(lse[h][~ok]))
-        np.testing.assert_allclose(lse[h][ok], lse_ref[ok], rtol=0, atol=2e-3 if w.dtype == "bf16" else 1e-5)
+        np.testing.assert_allclose(lse[h][ok], lse_ref[ok], rtol=0, atol=pu.LSE_TOL[w.dtype])
+
+
+@pytest.mark.parametrize("compensate", [True, False])
+@pytest.mark.parametrize("ck,density", [(400, 0.3), (37, 0.5), (250, 0.05)])
+def test_attention_packs_small_key_clusters(compensate, ck, density):
+    """Many small key clusters: most 32-row boxes are partial and one chunk
+    gathers boxes of several clusters (bf16 tensor-core path)."""
+    w = gen.MID.with_(heads=2, n=2000, d=128, n_centres=60, c_q=7, c_k=ck, iters=2,
+                      density=density)
+    L = gen.make_layer(w)
+    runs = [eo.pipeline(L.q[h], L.k[h], L.v[h], L.q_init[h], L.k_init[h], w.iters, w.density,
+                        compensate=compensate) for h in range(2)]
+    o, lse = _run_attention(L, runs, compensate)
+    for h, r in enumerate(runs):
+        ok = np.isfinite(r.lse)
+        pu.assert_attention_close(o[h][ok], r.o[ok], "bf16")
+        np.testing.assert_allclose(lse[h][ok], r.lse[ok], rtol=0, atol=pu.LSE_TOL["bf16"])
 
 
 # --------------------------------------------------------------------------- whole layer
