@@ -50,6 +50,15 @@ constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // move the running max only when it grows by > 2^8
+constexpr int kTableMax = 2048;   // block list / key offsets staged in shared memory up to this
+// Register split (setmaxnreg): warps 0-3 (producer, MMA issuer, 2 idle) drop
+// to kRegsLow, the two softmax warpgroups rise to kRegsHigh.  The sum stays
+// within the 168 registers x 384 threads the kernel is launched with; the
+// launcher checks the compiled count before every launch.
+constexpr int kRegsLow = 64;
+constexpr int kRegsHigh = 216;
+constexpr int kRegsLaunch = 168;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 // barrier slots
 constexpr int kBarKvFull = 0;   // + stage
@@ -77,7 +86,9 @@ struct Layout {
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBias = kV + kStages * kTileBytes;       // [stage][128] float
   static constexpr int kInfo = kBias + kStages * kChunk * 4;    // [stage] ChunkInfo
-  static constexpr int kBar = kInfo + kStages * 32;
+  static constexpr int kList = kInfo + kStages * 32;              // unit's exact key clusters
+  static constexpr int kKoff = kList + kTableMax * 4;             // slice's key offsets
+  static constexpr int kBar = kKoff + kTableMax * 4;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -111,12 +122,12 @@ struct Boxes {
   int compensate;
   int* status;
 
-  __device__ void init(const TcParams& p, int64_t h, int a) {
-    const int32_t* bo = p.blk_off + h * (int64_t)(p.Cq + 1);
-    list = p.blk_list + h * (int64_t)p.Cq * p.Ck;
-    koff = p.k_off + h * (int64_t)(p.Ck + 1);
-    e = bo[a];
-    e1 = bo[a + 1];
+  // list: the unit's exact key clusters [0, n); koff: the slice's key offsets.
+  __device__ void init(const TcParams& p, const int32_t* list_, int n, const int32_t* koff_) {
+    list = list_;
+    koff = koff_;
+    e = 0;
+    e1 = n;
     pos = end = 0;
     comp_next = 0;
     Ck = p.Ck;
@@ -225,63 +236,16 @@ __device__ __forceinline__ unsigned long long box_exp(const uint32_t (&v)[32],
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
-      const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+__device__ __forceinline__ void producer_role(
+    const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+    const CUtensorMap& tmKc, const CUtensorMap& tmVc, const TcParams& p, uint8_t* smem, int64_t h,
+    int a, int32_t row0, int ntiles, int lane, volatile int* abort) {
   using L = Layout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  const int64_t h = blockIdx.y;
-  const int64_t slot = blockIdx.x;
-  if (slot >= p.count[h]) return;
-  const int2 item = p.items[h * p.max_items + slot];
-  const int a = item.x;
-  const int32_t row0 = item.y;
-  const int32_t qend = p.q_off[h * (int64_t)(p.Cq + 1) + a + 1];
-  if (row0 < 0 || qend > p.Nq || row0 >= qend) {
-    if (threadIdx.x == 0) latch(p.status, EAR_ERR_DEVICE);
-    return;
-  }
-  const int rows_a = min(kTileRows, qend - row0);
-  const int rows_b = max(0, min(kTileRows, qend - row0 - kTileRows));
-  const int ntiles = rows_b > 0 ? 2 : 1;
-
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   float* bias = reinterpret_cast<float*>(smem + L::kBias);
   ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars[kBarKvFull + s], 1);
-      mbar_init(&bars[kBarKvEmpty + s], 1);
-    }
-    mbar_init(&bars[kBarQFull], 1);
-    mbar_init(&bars[kBarDrain], 1);
-    for (int t = 0; t < kTiles; ++t) {
-      mbar_init(&bars[kBarSFull + t], 1);
-      mbar_init(&bars[kBarPFull + t], kTileRows);
-      mbar_init(&bars[kBarODone + t], 1);
-    }
-    *abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+  {
+    {
     const uint8_t* exact_row = p.exact + (h * p.Cq + a) * (int64_t)p.Ck;
     const int32_t* koff = p.k_off + h * (int64_t)(p.Ck + 1);
     if (lane == 0) {
@@ -294,8 +258,24 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
           tma_load_2d(smem + L::kQ + t * L::kTileBytes + hf * L::kHalfBytes, &tmQ,
                       &bars[kBarQFull], 64 * hf, (int32_t)(h * p.Nq) + row0 + kTileRows * t);
     }
+    // Stage the unit's block list and the slice's key offsets in shared memory
+    // (the box walk below would otherwise chase them through L2 per block).
+    const int32_t* bo = p.blk_off + h * (int64_t)(p.Cq + 1);
+    const int32_t e0 = bo[a], nlist = bo[a + 1] - bo[a];
+    const int32_t* glist = p.blk_list + h * (int64_t)p.Cq * p.Ck + e0;
+    const int32_t* list = glist;
+    const int32_t* koff_t = koff;
+    if (nlist <= kTableMax && p.Ck + 1 <= kTableMax && nlist >= 0) {
+      int32_t* sl = reinterpret_cast<int32_t*>(smem + L::kList);
+      int32_t* sk = reinterpret_cast<int32_t*>(smem + L::kKoff);
+      for (int i = lane; i < nlist; i += 32) sl[i] = glist[i];
+      for (int i = lane; i <= p.Ck; i += 32) sk[i] = koff[i];
+      __syncwarp();
+      list = sl;
+      koff_t = sk;
+    }
     Boxes it;
-    it.init(p, h, a);
+    it.init(p, list, max(nlist, 0), koff_t);
     int32_t brow = 0;
     int bval = 0;
     bool bcomp = false;
@@ -306,25 +286,30 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
       if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
         break;
       issued = c + 1;
-      ChunkInfo ci;
-      ci.nbox = 0;
-      ci.comp = have && bcomp ? 1 : 0;
-      int32_t rows[kBoxes];
+      // up to four boxes of the same kind, held in registers (static indices)
+      const int comp = have && bcomp ? 1 : 0;
+      int nbox = 0;
+      int32_t r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+      int v0 = 0, v1 = 0, v2 = 0, v3 = 0;
       const int32_t comp_first = brow;
-      // up to four boxes of the same kind
-      while (have && ci.nbox < kBoxes && (bcomp ? 1 : 0) == ci.comp) {
-        rows[ci.nbox] = brow;
-        ci.valid[ci.nbox] = bval;
-        ++ci.nbox;
+#pragma unroll
+      for (int k = 0; k < kBoxes; ++k) {
+        if (!(have && (bcomp ? 1 : 0) == comp)) break;
+        if (k == 0) { r0 = brow; v0 = bval; }
+        if (k == 1) { r1 = brow; v1 = bval; }
+        if (k == 2) { r2 = brow; v2 = bval; }
+        if (k == 3) { r3 = brow; v3 = bval; }
+        nbox = k + 1;
         have = it.next(brow, bval, bcomp);
       }
-      if (ci.comp) {  // bias of the chunk's columns (centroids comp_first ...)
+      if (comp) {  // bias of the chunk's columns (centroids comp_first ...)
         for (int j = lane; j < kChunk; j += 32) {
           float bv = -INFINITY;
           const int bx = j / kBox;
-          if (bx < ci.nbox && (j % kBox) < ci.valid[bx]) {
+          const int vb = bx == 0 ? v0 : bx == 1 ? v1 : bx == 2 ? v2 : v3;
+          if (bx < nbox && (j % kBox) < vb) {
             const int b = comp_first + j;
-            const int32_t cnt = koff[b + 1] - koff[b];
+            const int32_t cnt = koff_t[b + 1] - koff_t[b];
             if (!exact_row[b] && cnt > 0) bv = __log2f((float)cnt);
           }
           bias[s * kChunk + j] = bv;
@@ -332,62 +317,94 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
       }
       __syncwarp();
       if (lane == 0) {
-        info[s] = ci;
-        if (ci.nbox == 0) {
+        ChunkInfo* ci = &info[s];
+        ci->nbox = nbox;
+        ci->comp = comp;
+        ci->valid[0] = v0;
+        ci->valid[1] = v1;
+        ci->valid[2] = v2;
+        ci->valid[3] = v3;
+        if (nbox == 0) {
           mbar_arrive(&bars[kBarKvFull + s]);  // end of the sequence
         } else {
-          mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * ci.nbox * kBox * D * 2);
-          const CUtensorMap* mk = ci.comp ? &tmKc : &tmK;
-          const CUtensorMap* mv = ci.comp ? &tmVc : &tmV;
-          const int32_t base = ci.comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
+          mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * nbox * kBox * D * 2);
+          const CUtensorMap* mk = comp ? &tmKc : &tmK;
+          const CUtensorMap* mv = comp ? &tmVc : &tmV;
+          const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
           uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
           uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
-          for (int bx = 0; bx < ci.nbox; ++bx)
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            if (bx >= nbox) break;
+            const int32_t rw = bx == 0 ? r0 : bx == 1 ? r1 : bx == 2 ? r2 : r3;
+#pragma unroll
             for (int hf = 0; hf < D / 64; ++hf) {
               tma_load_2d(kdst + hf * L::kHalfBytes + bx * kBox * 128, mk, &bars[kBarKvFull + s],
-                          64 * hf, base + rows[bx]);
+                          64 * hf, base + rw);
               tma_load_2d(vdst + hf * L::kHalfBytes + bx * kBox * 128, mv, &bars[kBarKvFull + s],
-                          64 * hf, base + rows[bx]);
+                          64 * hf, base + rw);
             }
+          }
         }
       }
       __syncwarp();
-      if (ci.nbox == 0) break;
+      if (nbox == 0) break;
     }
     if (*abort) {  // let issued loads land before the CTA exits
       mbar_wait_drain(&bars[kBarQFull], 0);
       for (int c = issued - 1; c >= 0 && c >= issued - kStages; --c)
         mbar_wait_drain(&bars[kBarKvFull + c % kStages], (c / kStages) & 1);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint32_t tmem, int ntiles,
+                                         volatile int* abort) {
+  using L = Layout<D>;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
+  {
+    {
+      // The whole warp runs this role and computes the operands (so they stay
+      // warp-uniform); one elected lane issues the MMAs and commits.
+      const bool leader = elect_one();
       const uint32_t idesc_pv = idesc_bf16(128, D, true);
       auto issue_qk = [&](int t, int s, int n) {
         const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
         const uint32_t qb = smem_u32(smem + L::kQ + t * L::kTileBytes);
         const uint32_t kb = smem_u32(smem + L::kK + s * L::kTileBytes);
+        const uint64_t qd = desc_sw128(qb, 16, 1024), kd = desc_sw128(kb, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * L::kHalfBytes + (kk % 4) * 32;
-          mma_ss(tmem + kTileRows * t, desc_sw128(qb + off, 16, 1024),
-                 desc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * L::kHalfBytes + (kk % 4) * 32) >> 4;
+          if (leader) mma_ss(tmem + kTileRows * t, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int s, int n, bool first) {
         const uint32_t vb = smem_u32(smem + L::kV + s * L::kTileBytes);
-        for (int kk = 0; kk < n / 16; ++kk)
-          mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kk * 8,
-                 desc_sw128(vb + kk * 2048, L::kHalfBytes, 1024), idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
+        const uint64_t vd = desc_sw128(vb, L::kHalfBytes, 1024);
+        const int nk = n / 16;
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          if (kk < nk && leader)
+            mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kk * 8,
+                   vd + ((kk * 2048) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
       };
-      bool ok = mbar_wait(&bars[kBarQFull], 0, abort) && mbar_wait(&bars[kBarKvFull], 0, abort);
+      auto commit = [&](uint64_t* bar) {
+        if (leader) mma_commit(bar);
+        __syncwarp();
+      };
+      bool ok = mbar_wait_warp(&bars[kBarQFull], 0, abort) &&
+                mbar_wait_warp(&bars[kBarKvFull], 0, abort);
       int n_cur = ok ? info[0].nbox * kBox : 0;
       if (ok && n_cur > 0) {
         tc_fence_after();
         for (int t = 0; t < ntiles; ++t) {
           issue_qk(t, 0, n_cur);
-          mma_commit(&bars[kBarSFull + t]);
+          commit(&bars[kBarSFull + t]);
         }
       }
       for (int c = 0; ok && n_cur > 0; ++c) {
@@ -395,31 +412,41 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
         const int s2 = (c + 1) % kStages;
         int n_nxt = 0;
         for (int t = 0; t < ntiles && ok; ++t) {
-          ok = mbar_wait(&bars[kBarPFull + t], c & 1, abort);
+          ok = mbar_wait_warp(&bars[kBarPFull + t], c & 1, abort);
           if (!ok) break;
           tc_fence_after();
           issue_pv(t, s, n_cur, c == 0);
-          mma_commit(&bars[kBarODone + t]);
-          if (t == ntiles - 1) mma_commit(&bars[kBarKvEmpty + s]);
+          commit(&bars[kBarODone + t]);
+          if (t == ntiles - 1) commit(&bars[kBarKvEmpty + s]);
           if (t == 0) {
-            ok = mbar_wait(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
+            ok = mbar_wait_warp(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
             if (!ok) break;
             n_nxt = info[s2].nbox * kBox;
             tc_fence_after();
           }
           if (n_nxt > 0) {
             issue_qk(t, s2, n_nxt);
-            mma_commit(&bars[kBarSFull + t]);
+            commit(&bars[kBarSFull + t]);
           }
         }
         n_cur = n_nxt;
       }
       // every MMA issued above has finished before TMEM is released
-      mma_commit(&bars[kBarDrain]);
+      commit(&bars[kBarDrain]);
       mbar_wait_drain(&bars[kBarDrain], 0);
     }
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------------- softmax
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, uint32_t tmem,
+                                             int64_t h, int32_t row0, int rows_a, int rows_b,
+                                             int ntiles, int warp, int lane, volatile int* abort) {
+  using L = Layout<D>;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  float* bias = reinterpret_cast<float*>(smem + L::kBias);
+  ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
+  {
     const int t = (warp - 4) / 4;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row within the tile = TMEM lane
@@ -548,13 +575,86 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
     }
   }
 
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+      const __grid_constant__ CUtensorMap tmVc, const TcParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int64_t h = blockIdx.y;
+  const int64_t slot = blockIdx.x;
+  if (slot >= p.count[h]) return;
+  const int2 item = p.items[h * p.max_items + slot];
+  const int a = item.x;
+  const int32_t row0 = item.y;
+  const int32_t qend = p.q_off[h * (int64_t)(p.Cq + 1) + a + 1];
+  if (row0 < 0 || qend > p.Nq || row0 >= qend) {
+    if (threadIdx.x == 0) latch(p.status, EAR_ERR_DEVICE);
+    return;
+  }
+  const int rows_a = min(kTileRows, qend - row0);
+  const int rows_b = max(0, min(kTileRows, qend - row0 - kTileRows));
+  const int ntiles = rows_b > 0 ? 2 : 1;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* bias = reinterpret_cast<float*>(smem + L::kBias);
+  ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[kBarKvFull + s], 1);
+      mbar_init(&bars[kBarKvEmpty + s], 1);
+    }
+    mbar_init(&bars[kBarQFull], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&bars[kBarSFull + t], 1);
+      mbar_init(&bars[kBarPFull + t], kTileRows);
+      mbar_init(&bars[kBarODone + t], 1);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Each role ends with its own teardown (a CTA-wide bar.sync, then warp 0
+  // frees TMEM), so no code runs under both register budgets.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsLow));
+    if (warp == 0) {
+      producer_role<D>(tmQ, tmK, tmV, tmKc, tmVc, p, smem, h, a, row0, ntiles, lane, abort);
+    } else if (warp == 1) {
+      mma_role<D>(p, smem, tmem, ntiles, abort);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 0;" ::: "memory");
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+      if (lane == 0 && *abort) latch(p.status, EAR_ERR_TIMEOUT);
+    }
+    return;
   }
-  if (threadIdx.x == 0 && *abort) latch(p.status, EAR_ERR_TIMEOUT);
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsHigh));
+  softmax_role<D>(p, smem, tmem, h, row0, rows_a, rows_b, ntiles, warp, lane, abort);
+  tc_fence_before();
+  asm volatile("bar.sync 0;" ::: "memory");
 }
 
 __global__ void at_centroids_bf16(const float* __restrict__ kc, const float* __restrict__ vc,
@@ -639,6 +739,11 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
   p.lse = a.lse;
   p.status = device_status_word();
   EAR_CUDA(cudaFuncSetAttribute(at_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  // setmaxnreg.inc waits until the block's launch registers cover the split:
+  // refuse to launch a build whose allocation does not.
+  cudaFuncAttributes fa;
+  EAR_CUDA(cudaFuncGetAttributes(&fa, at_tc<D>));
+  if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh) return EAR_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)max_items, (unsigned)a.bh);
   at_tc<D><<<grid, kThreads, L::kBytes, s>>>(mq, mk, mv, mkc, mvc, p);
   return after_launch();
