@@ -17,16 +17,16 @@
 //               ring.  It publishes each stage's chunk descriptor (box count,
 //               valid rows per box, centroid or not, bias) in shared memory
 //               and ends the sequence with an empty descriptor.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T into TMEM, then
+//   warp 1      MMA issuer (one elected lane of the warp): S_t = Q_t K^T into TMEM, then
 //               O_t += P_t V with P_t read from TMEM.  Issue order
 //               QK_A(c) QK_B(c) | PV_A(c) QK_A(c+1) PV_B(c) QK_B(c+1) | ...
 //               so one tile's softmax overlaps the other tile's MMAs.
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread
 //               per query row (= TMEM lane).  Online softmax in base 2 on the
-//               raw scores: the max pass is one compare per score, the
-//               exponent argument one packed FMA per score pair; the running
-//               max only moves (and O is rescaled in TMEM) when it grows by
-//               more than 2^8.
+//               raw scores: an exact chunk is read from TMEM once (max, then
+//               exponent, from registers); the exponent argument is one packed
+//               FMA per score pair; the running max only moves (and O is
+//               rescaled in TMEM) when it grows by more than 2^8.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512);
 // P_t (bf16 pairs) overwrites the first half of S_t.
 #include <mutex>
@@ -235,6 +235,27 @@ __device__ __forceinline__ unsigned long long box_exp(const uint32_t (&v)[32],
   return sum;
 }
 
+// box_exp with one shift pair for every column (exact box)
+__device__ __forceinline__ unsigned long long box_exp_c(const uint32_t (&v)[32],
+                                                        unsigned long long sh,
+                                                        unsigned long long scale2, int valid,
+                                                        uint32_t (&pk)[16]) {
+  unsigned long long sum0 = 0, sum1 = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const unsigned long long z = fma2(pack2(v[j], v[j + 1]), scale2, sh);
+    float p0 = ex2(lo_f(z)), p1 = ex2(hi_f(z));
+    if (valid < 32) {
+      p0 = j < valid ? p0 : 0.f;
+      p1 = j + 1 < valid ? p1 : 0.f;
+    }
+    const unsigned long long pr = pack2(__float_as_uint(p0), __float_as_uint(p1));
+    if (j & 2) sum1 = add2(sum1, pr); else sum0 = add2(sum0, pr);
+    pk[j / 2] = pack_bf16x2(p0, p1);
+  }
+  return add2(sum0, sum1);
+}
+
 template <int D>
 __device__ __forceinline__ void producer_role(
     const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
@@ -248,7 +269,8 @@ __device__ __forceinline__ void producer_role(
     {
     const uint8_t* exact_row = p.exact + (h * p.Cq + a) * (int64_t)p.Ck;
     const int32_t* koff = p.k_off + h * (int64_t)(p.Ck + 1);
-    if (lane == 0) {
+    const bool leader = elect_one();  // issues the TMA copies (operands stay warp-uniform)
+    if (leader) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -316,7 +338,7 @@ __device__ __forceinline__ void producer_role(
         }
       }
       __syncwarp();
-      if (lane == 0) {
+      if (leader) {
         ChunkInfo* ci = &info[s];
         ci->nbox = nbox;
         ci->comp = comp;
@@ -324,21 +346,23 @@ __device__ __forceinline__ void producer_role(
         ci->valid[1] = v1;
         ci->valid[2] = v2;
         ci->valid[3] = v3;
-        if (nbox == 0) {
+        if (nbox == 0)
           mbar_arrive(&bars[kBarKvFull + s]);  // end of the sequence
-        } else {
+        else
           mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * nbox * kBox * D * 2);
-          const CUtensorMap* mk = comp ? &tmKc : &tmK;
-          const CUtensorMap* mv = comp ? &tmVc : &tmV;
-          const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
-          uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
-          uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
+      }
+      {
+        const CUtensorMap* mk = comp ? &tmKc : &tmK;
+        const CUtensorMap* mv = comp ? &tmVc : &tmV;
+        const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
+        uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
+        uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
 #pragma unroll
-          for (int bx = 0; bx < kBoxes; ++bx) {
-            if (bx >= nbox) break;
-            const int32_t rw = bx == 0 ? r0 : bx == 1 ? r1 : bx == 2 ? r2 : r3;
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          const int32_t rw = bx == 0 ? r0 : bx == 1 ? r1 : bx == 2 ? r2 : r3;
 #pragma unroll
-            for (int hf = 0; hf < D / 64; ++hf) {
+          for (int hf = 0; hf < D / 64; ++hf) {
+            if (bx < nbox && leader) {
               tma_load_2d(kdst + hf * L::kHalfBytes + bx * kBox * 128, mk, &bars[kBarKvFull + s],
                           64 * hf, base + rw);
               tma_load_2d(vdst + hf * L::kHalfBytes + bx * kBox * 128, mv, &bars[kBarKvFull + s],
@@ -473,54 +497,83 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
         if (!ok) break;
         tc_fence_after();
         const float* bs = bias + s * kChunk;
-        // pass 1: chunk max (scaled)
-        float mx = -INFINITY;
-        for (int bx = 0; bx < nbox; bx += 2) {
-          uint32_t va[32], vb[32];
-          const bool has_b = bx + 1 < nbox;
-          tmem_ld32(tS + 32 * bx, va);
-          if (has_b) tmem_ld32(tS + 32 * (bx + 1), vb);
+        bool resc = false;
+        float corr = 1.f, m_use = m;
+        if (!comp) {
+          // exact chunk: one TMEM trip for all four boxes (unused boxes have
+          // valid = 0), max and exponent from registers
+          const int v0 = ci->valid[0], v1 = ci->valid[1], v2 = ci->valid[2], v3 = ci->valid[3];
+          uint32_t x0[32], x1[32], x2[32], x3[32];
+          tmem_ld32(tS, x0);
+          tmem_ld32(tS + 32, x1);
+          tmem_ld32(tS + 64, x2);
+          tmem_ld32(tS + 96, x3);
           tmem_ld_wait();
-          const int v0 = ci->valid[bx], v1 = has_b ? ci->valid[bx + 1] : 0;
-          if (!comp) {
-            mx = fmaxf(mx, box_max_raw(va, v0) * scale);
-            if (has_b) mx = fmaxf(mx, box_max_raw(vb, v1) * scale);
-          } else {
+          const float mx = fmaxf(fmaxf(box_max_raw(x0, v0), box_max_raw(x1, v1)),
+                                 fmaxf(box_max_raw(x2, v2), box_max_raw(x3, v3))) * scale;
+          if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
+            if (m != -INFINITY) {
+              resc = true;
+              corr = ex2(m - mx);
+            }
+            m_use = mx;
+          }
+          if (resc) lsum = pack2(__float_as_uint(lo_f(lsum) * corr), __float_as_uint(hi_f(lsum) * corr));
+          const float neg = m_use == -INFINITY ? 0.f : -m_use;
+          const unsigned long long n2 = pack2(__float_as_uint(neg), __float_as_uint(neg));
+          const bool none = m_use == -INFINITY;  // every score -inf: p = 0
+          uint32_t pk[16];
+          lsum = add2(lsum, box_exp_c(x0, n2, scale2, none ? 0 : v0, pk));
+          tmem_st16(tS, pk);
+          if (nbox > 1) {
+            lsum = add2(lsum, box_exp_c(x1, n2, scale2, none ? 0 : v1, pk));
+            tmem_st16(tS + 16, pk);
+          }
+          if (nbox > 2) {
+            lsum = add2(lsum, box_exp_c(x2, n2, scale2, none ? 0 : v2, pk));
+            tmem_st16(tS + 32, pk);
+          }
+          if (nbox > 3) {
+            lsum = add2(lsum, box_exp_c(x3, n2, scale2, none ? 0 : v3, pk));
+            tmem_st16(tS + 48, pk);
+          }
+        } else {
+          // centroid chunk, pass 1: chunk max (scaled, with the bias)
+          float mx = -INFINITY;
+          for (int bx = 0; bx < nbox; bx += 2) {
+            uint32_t va[32], vb[32];
+            const bool has_b = bx + 1 < nbox;
+            tmem_ld32(tS + 32 * bx, va);
+            if (has_b) tmem_ld32(tS + 32 * (bx + 1), vb);
+            tmem_ld_wait();
+            const int v0 = ci->valid[bx], v1 = has_b ? ci->valid[bx + 1] : 0;
             mx = fmaxf(mx, box_max_bias(va, bs + 32 * bx, scale, v0));
             if (has_b) mx = fmaxf(mx, box_max_bias(vb, bs + 32 * (bx + 1), scale, v1));
           }
-        }
-        float m_use = m, corr = 1.f;
-        bool resc = false;
-        if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
-          if (m != -INFINITY) {
-            resc = true;
-            corr = ex2(m - mx);
+          if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
+            if (m != -INFINITY) {
+              resc = true;
+              corr = ex2(m - mx);
+            }
+            m_use = mx;
           }
-          m_use = mx;
-        }
-        if (resc) lsum = pack2(__float_as_uint(lo_f(lsum) * corr), __float_as_uint(hi_f(lsum) * corr));
-        // pass 2: P = 2^(scaled score - m_use) into the first half of S
-        const float neg = m_use == -INFINITY ? 0.f : -m_use;  // all scores -inf: p = 0 below
-        for (int bx = 0; bx < nbox; ++bx) {
-          uint32_t v[32];
-          tmem_ld32(tS + 32 * bx, v);
-          tmem_ld_wait();
-          unsigned long long sh[16];
-          if (!comp) {
-            const unsigned long long n2 = pack2(__float_as_uint(neg), __float_as_uint(neg));
-#pragma unroll
-            for (int j = 0; j < 16; ++j) sh[j] = n2;
-          } else {
+          if (resc) lsum = pack2(__float_as_uint(lo_f(lsum) * corr), __float_as_uint(hi_f(lsum) * corr));
+          // centroid chunk, pass 2: P = 2^(scaled score + bias - m_use) into the first half of S
+          const float neg = m_use == -INFINITY ? 0.f : -m_use;  // all scores -inf: p = 0 below
+          for (int bx = 0; bx < nbox; ++bx) {
+            uint32_t v[32];
+            tmem_ld32(tS + 32 * bx, v);
+            tmem_ld_wait();
+            unsigned long long sh[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               sh[j] = pack2(__float_as_uint(bs[32 * bx + 2 * j] + neg),
                             __float_as_uint(bs[32 * bx + 2 * j + 1] + neg));
+            const int valid = m_use == -INFINITY ? 0 : ci->valid[bx];
+            uint32_t pk[16];
+            lsum = add2(lsum, box_exp(v, sh, scale2, valid, pk));
+            tmem_st16(tS + 16 * bx, pk);
           }
-          const int valid = m_use == -INFINITY ? 0 : ci->valid[bx];
-          uint32_t pk[16];
-          lsum = add2(lsum, box_exp(v, sh, scale2, valid, pk));
-          tmem_st16(tS + 16 * bx, pk);
         }
         tmem_st_wait();
         if (__any_sync(0xffffffffu, resc)) {
