@@ -302,18 +302,17 @@ __device__ __forceinline__ void producer_role(
     int bval = 0;
     bool bcomp = false;
     bool have = it.next(brow, bval, bcomp);  // the box that opens the next chunk
-    int issued = 0;
-    for (int c = 0;; ++c) {
-      const int s = c % kStages;
-      if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
-        break;
-      issued = c + 1;
-      // up to four boxes of the same kind, held in registers (static indices)
-      const int comp = have && bcomp ? 1 : 0;
-      int nbox = 0;
-      int32_t r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-      int v0 = 0, v1 = 0, v2 = 0, v3 = 0;
-      const int32_t comp_first = brow;
+    // The next chunk: up to four boxes of the same kind, held in registers
+    // (static indices).  It is gathered while the ring slot is still busy.
+    int comp = 0, nbox = 0;
+    int32_t r0 = 0, r1 = 0, r2 = 0, r3 = 0, comp_first = 0;
+    int v0 = 0, v1 = 0, v2 = 0, v3 = 0;
+    auto gather = [&]() {
+      comp = have && bcomp ? 1 : 0;
+      nbox = 0;
+      r0 = r1 = r2 = r3 = 0;
+      v0 = v1 = v2 = v3 = 0;
+      comp_first = brow;
 #pragma unroll
       for (int k = 0; k < kBoxes; ++k) {
         if (!(have && (bcomp ? 1 : 0) == comp)) break;
@@ -324,6 +323,14 @@ __device__ __forceinline__ void producer_role(
         nbox = k + 1;
         have = it.next(brow, bval, bcomp);
       }
+    };
+    gather();
+    int issued = 0;
+    for (int c = 0;; ++c) {
+      const int s = c % kStages;
+      if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
+        break;
+      issued = c + 1;
       if (comp) {  // bias of the chunk's columns (centroids comp_first ...)
         for (int j = lane; j < kChunk; j += 32) {
           float bv = -INFINITY;
@@ -373,6 +380,7 @@ __device__ __forceinline__ void producer_role(
       }
       __syncwarp();
       if (nbox == 0) break;
+      gather();
     }
     if (*abort) {  // let issued loads land before the CTA exits
       mbar_wait_drain(&bars[kBarQFull], 0);
