@@ -18,14 +18,17 @@
 //                the rounding margin of the running minimum.  One candidate
 //                = a certain label; 2-4 candidates go to an fp64 decision
 //                among them; more (or a row / centroid without an exact fp16
-//                copy) go to a full fp64 decision.  Certain rows whose label
-//                changed are listed as moves.
-//   km_pick64    fp64 distances of the 2-4 candidates of a listed row, in the
-//                order sum_k (x_k - c_k)^2 k = 0..d-1 (ties to the lowest
-//                index), then the row's move.
-//   km_refine64  the same over all C centroids for the rows that need it.
-//   km_moves     sums[new] += x, sums[old] -= x, counts likewise (vector fp32
-//                atomics): after the first iteration only moved rows cost work.
+//                copy) go to a full fp64 decision.  Each row's outcome is a
+//                byte of its own (moved / pick with n candidates / full), the
+//                candidates and the old label go to per-row slots: plain
+//                coalesced stores, no list counters.
+//   km_resolve   one warp per 32-row window of those bytes: moves (sums[new]
+//                += x, sums[old] -= x, counts likewise, vector fp32 atomics),
+//                picks (fp64 distances of the 2-4 candidates in the order
+//                sum_k (x_k - c_k)^2, k = 0..d-1, ties to the lowest index;
+//                eight rows per warp) and full decisions (the same over all C
+//                centroids, four per lane at a time), each followed by its
+//                move.  After the first iteration only moved rows cost atomics.
 //   km_finalize  centroid = sum / count (empty clusters keep theirs), and the
 //                fp16 copy / norms / max norm for the next iteration.
 //
@@ -86,18 +89,11 @@ struct KLayout {
   static constexpr int kBytes = kMisc + 16 + 1024;
 };
 
-struct Move {
-  int64_t row;
-  int32_t from;
-  int32_t to;
-};
-
-struct Pick {
-  int64_t row;
-  int32_t n;
-  int32_t cand[4];
-  int32_t pad;
-};
+// per-row outcome byte: bits 0-1 kind, bits 2-4 pick candidate count
+constexpr uint8_t kKindNone = 0;    // certain, label unchanged
+constexpr uint8_t kKindMove = 1;    // certain, label changed (old label in `from`)
+constexpr uint8_t kKindPick = 2;    // 2-4 candidates in `cand`
+constexpr uint8_t kKindFull = 3;    // fp64 decision over every centroid
 
 struct KmTcParams {
   const float* xnorm;       // [BH*N]
@@ -105,12 +101,9 @@ struct KmTcParams {
   const float* cmax;        // [BH]
   const int* cbad;          // [BH] a centroid of the slice has no finite fp16 copy
   int32_t* labels;          // [BH*N]
-  int64_t* refine_rows;     // rows for the full fp64 decision
-  unsigned long long* refine_count;
-  struct Pick* picks;       // rows with 2-4 candidates
-  unsigned long long* pick_count;
-  Move* moves;
-  unsigned long long* move_count;
+  uint8_t* kind;            // [BH*N] outcome byte
+  int4* cand;               // [BH*N] pick candidates
+  int32_t* from;            // [BH*N] old label of a moved row
   int64_t N;
   int C, C_pad, first;
   int c_box;  // rows per centroid TMA box (min(256, C_pad))
@@ -121,31 +114,35 @@ __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// Appends one entry per active lane with a single atomic per warp.
-__device__ __forceinline__ unsigned long long warp_append(unsigned long long* counter, bool want) {
-  const unsigned mask = __ballot_sync(0xffffffffu, want);
-  const int lane = threadIdx.x & 31;
-  unsigned long long base = 0;
-  const int leader = mask ? __ffs(mask) - 1 : 0;
-  if (mask && lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(mask));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  return base + __popc(mask & ((1u << lane) - 1u));
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
-// min over 32 columns of d~ = cn - 2 v, four independent chains
+// min over 32 columns of d~ = cn - 2 v, four independent chains of
+// three-input minima; the norms come in as 16-byte loads
 __device__ __forceinline__ float group_min(const uint32_t (&v)[32], const float* cn) {
   const unsigned long long m2 = 0xC0000000C0000000ull;  // (-2.f, -2.f)
-  const unsigned long long* c2 = reinterpret_cast<const unsigned long long*>(cn);
+  const float4* c4 = reinterpret_cast<const float4*>(cn);
   float m[4] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000),
                 __int_as_float(0x7f800000), __int_as_float(0x7f800000)};
 #pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    const unsigned long long vv = (unsigned long long)v[k] | ((unsigned long long)v[k + 1] << 32);
-    unsigned long long dd;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dd) : "l"(vv), "l"(m2), "l"(c2[k / 2]));
-    const int a = (k / 2) & 1;
-    m[2 * a] = fminf(m[2 * a], __uint_as_float((uint32_t)dd));
-    m[2 * a + 1] = fminf(m[2 * a + 1], __uint_as_float((uint32_t)(dd >> 32)));
+  for (int k = 0; k < 32; k += 4) {
+    const float4 cc = c4[k / 4];
+    const unsigned long long c01 =
+        (unsigned long long)__float_as_uint(cc.x) | ((unsigned long long)__float_as_uint(cc.y) << 32);
+    const unsigned long long c23 =
+        (unsigned long long)__float_as_uint(cc.z) | ((unsigned long long)__float_as_uint(cc.w) << 32);
+    const unsigned long long v01 = (unsigned long long)v[k] | ((unsigned long long)v[k + 1] << 32);
+    const unsigned long long v23 =
+        (unsigned long long)v[k + 2] | ((unsigned long long)v[k + 3] << 32);
+    unsigned long long d01, d23;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d01) : "l"(v01), "l"(m2), "l"(c01));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d23) : "l"(v23), "l"(m2), "l"(c23));
+    const int a = (k / 4) & 3;
+    m[a] = min3f(m[a], __uint_as_float((uint32_t)d01), __uint_as_float((uint32_t)(d01 >> 32)));
+    m[a] = min3f(m[a], __uint_as_float((uint32_t)d23), __uint_as_float((uint32_t)(d23 >> 32)));
   }
   return fminf(fminf(m[0], m[1]), fminf(m[2], m[3]));
 }
@@ -387,30 +384,19 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
           }
         }
         full = full || keep == 0 || keep > 4;
-        bool moved = false, pick = false;
-        int old = -1;
         if (valid) {
-          old = p.first ? -1 : p.labels[g];
+          const int old = p.first ? -1 : p.labels[g];
+          uint8_t kind = kKindFull;
           if (!full && keep == 1) {
             p.labels[g] = kc[0];
-            moved = kc[0] != old;
-          } else {
-            pick = !full;
+            kind = kc[0] != old ? kKindMove : kKindNone;
+            if (kind == kKindMove) p.from[g] = old;
+          } else if (!full) {
+            kind = (uint8_t)(kKindPick | (keep << 2));
+            p.cand[g] = make_int4(kc[0], kc[1], kc[2], kc[3]);
           }
+          p.kind[g] = kind;
         }
-        const unsigned long long pr = warp_append(p.refine_count, valid && full);
-        if (valid && full) p.refine_rows[pr] = g;
-        const unsigned long long pp = warp_append(p.pick_count, pick);
-        if (pick) {
-          Pick e;
-          e.row = g;
-          e.n = keep;
-          e.cand[0] = kc[0]; e.cand[1] = kc[1]; e.cand[2] = kc[2]; e.cand[3] = kc[3];
-          e.pad = 0;
-          p.picks[pp] = e;
-        }
-        const unsigned long long pm = warp_append(p.move_count, moved);
-        if (moved) p.moves[pm] = Move{g, old, kc[0]};
       }
     }
   }
@@ -500,147 +486,147 @@ __global__ void km_cprep(const float* __restrict__ cent, __half* __restrict__ ch
            D, c < C);
 }
 
-// exact fp64 argmin for the listed rows, then their moves
+// sums[to] += x, sums[from] -= x (no old cluster when !has_from) for one row;
+// the `gs` lanes of a group (rank `u`) take 4-value slices.
 template <typename T, int D>
-__global__ void km_refine64(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
-                            int C, int32_t* __restrict__ labels, int first,
-                            const int64_t* __restrict__ rows,
-                            const unsigned long long* __restrict__ count,
-                            float* __restrict__ sums, int32_t* __restrict__ cnt) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t total = (int64_t)*count;
-  for (int64_t e = warp; e < total; e += nw) {
-    const int64_t g = rows[e];
-    const int64_t h = g / N;
-    const T* x = X + g * D;
-    const float* ch = cent + h * (int64_t)C * D;
-    double best = __longlong_as_double(0x7ff0000000000000ll);
-    int bidx = 0;
-    for (int c = lane; c < C; c += 32) {
-      const float* cc = ch + (int64_t)c * D;
-      double dist = 0.0;
-      for (int k = 0; k < D; ++k) {
-        const double diff = __dsub_rn((double)Elem<T>::load(x, k), (double)cc[k]);
-        dist = __dadd_rn(dist, __dmul_rn(diff, diff));
-      }
-      if (dist < best) {
-        best = dist;
-        bidx = c;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-      if (ob < best || (ob == best && oi < bidx)) {
-        best = ob;
-        bidx = oi;
-      }
-    }
-    const int old = first ? -1 : labels[g];
-    __syncwarp();
-    if (lane == 0) labels[g] = bidx;
-    if (bidx != old) {
-      for (int k = lane * 4; k < D; k += 128) {
-        const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
-                                     Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
-        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + bidx) * D + k), v);
-        if (old >= 0)
-          atomicAdd(reinterpret_cast<float4*>(sums + (h * C + old) * D + k),
-                    make_float4(-v.x, -v.y, -v.z, -v.w));
-      }
-      if (lane == 0) {
-        atomicAdd(cnt + h * C + bidx, 1);
-        if (old >= 0) atomicAdd(cnt + h * C + old, -1);
-      }
+__device__ __forceinline__ void move_row(const T* __restrict__ x, float* __restrict__ sums,
+                                         int32_t* __restrict__ cnt, int64_t hc_to,
+                                         int64_t hc_from, bool has_from, int u, int gs) {
+  for (int k = u * 4; k < D; k += 4 * gs) {
+    const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
+                                 Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
+    atomicAdd(reinterpret_cast<float4*>(sums + hc_to * D + k), v);
+    if (has_from)
+      atomicAdd(reinterpret_cast<float4*>(sums + hc_from * D + k),
+                make_float4(-v.x, -v.y, -v.z, -v.w));
+  }
+  if (u == 0) {
+    atomicAdd(cnt + hc_to, 1);
+    if (has_from) atomicAdd(cnt + hc_from, -1);
+  }
+}
+
+// fp64 squared distance in the oracle's order: sum_k (x_k - c_k)^2, k = 0..D-1,
+// one rounding per operation (no contraction)
+template <typename T, int D>
+__device__ __forceinline__ double dist64(const T* __restrict__ x, const float* __restrict__ c) {
+  double dist = 0.0;
+  for (int k = 0; k < D; ++k) {
+    const double diff = __dsub_rn((double)Elem<T>::load(x, k), (double)c[k]);
+    dist = __dadd_rn(dist, __dmul_rn(diff, diff));
+  }
+  return dist;
+}
+
+// (best, index) across the lanes xor-reachable with offsets < `width`; ties
+// go to the lower index
+__device__ __forceinline__ void argmin_lanes(double& best, int& bidx, int width) {
+  for (int off = width / 2; off >= 1; off >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+    if (ob < best || (ob == best && oi < bidx)) {
+      best = ob;
+      bidx = oi;
     }
   }
 }
 
-// fp64 decision among a row's 2-4 candidates (lane u takes candidate u),
-// then the move.
+// Resolves every row decided in km_tc: one warp per window of 32 rows.
 template <typename T, int D>
-__global__ void km_pick64(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
-                          int C, int32_t* __restrict__ labels, int first,
-                          const Pick* __restrict__ picks,
-                          const unsigned long long* __restrict__ count,
-                          float* __restrict__ sums, int32_t* __restrict__ cnt) {
+__global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
+                           int C, int64_t rows, int32_t* __restrict__ labels, int first,
+                           const uint8_t* __restrict__ kind, const int4* __restrict__ cand,
+                           const int32_t* __restrict__ from, float* __restrict__ sums,
+                           int32_t* __restrict__ cnt) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t total = (int64_t)*count;
-  for (int64_t e = warp; e < total; e += nw) {
-    const Pick pk = picks[e];
-    const int64_t g = pk.row;
-    const int64_t h = g / N;
-    const T* x = X + g * D;
-    double best = __longlong_as_double(0x7ff0000000000000ll);
-    int bidx = C;
-    if (lane < pk.n) {
-      const int c = pk.cand[lane];
-      const float* cc = cent + (h * C + c) * (int64_t)D;
-      double dist = 0.0;
-      for (int k = 0; k < D; ++k) {
-        const double diff = __dsub_rn((double)Elem<T>::load(x, k), (double)cc[k]);
-        dist = __dadd_rn(dist, __dmul_rn(diff, diff));
-      }
-      best = dist;
-      bidx = c;
+  const int64_t nwin = (rows + 31) / 32;
+  for (int64_t win = warp; win < nwin; win += nw) {
+    const int64_t gl = win * 32 + lane;
+    const uint8_t kd = gl < rows ? kind[gl] : kKindNone;
+    // moves of certain rows
+    unsigned m = __ballot_sync(0xffffffffu, (kd & 3) == kKindMove);
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1;
+      const int64_t g = win * 32 + i;
+      const int64_t h = g / N;
+      const int old = from[g];
+      move_row<T, D>(X + g * D, sums, cnt, h * C + labels[g], h * C + old, old >= 0, lane, 32);
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-      if (ob < best || (ob == best && oi < bidx)) {
-        best = ob;
-        bidx = oi;
+    // picks: eight rows at a time, lane 4r + u takes candidate u of row r
+    unsigned pm = __ballot_sync(0xffffffffu, (kd & 3) == kKindPick);
+    while (pm) {
+      int myrow = -1;
+      for (int r = 0; r < 8 && pm; ++r) {  // the r-th of the next eight rows
+        const int i = __ffs(pm) - 1;
+        pm &= pm - 1;
+        if ((lane >> 2) == r) myrow = i;
       }
-    }
-    const int old = first ? -1 : labels[g];
-    __syncwarp();
-    if (lane == 0) labels[g] = bidx;
-    if (bidx != old) {
-      for (int k = lane * 4; k < D; k += 128) {
-        const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
-                                     Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
-        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + bidx) * D + k), v);
-        if (old >= 0)
-          atomicAdd(reinterpret_cast<float4*>(sums + (h * C + old) * D + k),
-                    make_float4(-v.x, -v.y, -v.z, -v.w));
+      const int r = lane >> 2, u = lane & 3;
+      const bool live = myrow >= 0;
+      const int64_t g = win * 32 + (live ? myrow : 0);
+      const int64_t h = g / N;
+      const T* x = X + g * D;
+      double best = __longlong_as_double(0x7ff0000000000000ll);
+      int bidx = C;
+      if (live) {
+        const int n = (kind[g] >> 2) & 7;
+        if (u < n) {
+          const int4 cc = cand[g];
+          const int c = u == 0 ? cc.x : u == 1 ? cc.y : u == 2 ? cc.z : cc.w;
+          best = dist64<T, D>(x, cent + (h * C + c) * (int64_t)D);
+          bidx = c;
+        }
       }
-      if (lane == 0) {
-        atomicAdd(cnt + h * C + bidx, 1);
-        if (old >= 0) atomicAdd(cnt + h * C + old, -1);
+      argmin_lanes(best, bidx, 4);
+      int old = -1;
+      if (live) old = first ? -1 : labels[g];
+      __syncwarp();
+      if (live && u == 0) labels[g] = bidx;
+      if (live && bidx != old)
+        move_row<T, D>(x, sums, cnt, h * C + bidx, h * C + old, old >= 0, u, 4);
+      (void)r;
+    }
+    // full fp64 decisions: a lane carries centroids c, c+32, c+64, c+96 (four
+    // independent chains, compared in increasing index order)
+    unsigned fm = __ballot_sync(0xffffffffu, (kd & 3) == kKindFull);
+    while (fm) {
+      const int i = __ffs(fm) - 1;
+      fm &= fm - 1;
+      const int64_t g = win * 32 + i;
+      const int64_t h = g / N;
+      const T* x = X + g * D;
+      const float* ch = cent + h * (int64_t)C * D;
+      double best = __longlong_as_double(0x7ff0000000000000ll);
+      int bidx = 0;
+      for (int c0 = lane; c0 < C; c0 += 128) {
+        const int c1 = c0 + 32, c2 = c0 + 64, c3 = c0 + 96;
+        const float* p0 = ch + (int64_t)c0 * D;
+        const float* p1 = ch + (int64_t)(c1 < C ? c1 : c0) * D;
+        const float* p2 = ch + (int64_t)(c2 < C ? c2 : c0) * D;
+        const float* p3 = ch + (int64_t)(c3 < C ? c3 : c0) * D;
+        double d0 = 0.0, d1 = 0.0, d2 = 0.0, d3 = 0.0;
+        for (int k = 0; k < D; ++k) {
+          const double xv = (double)Elem<T>::load(x, k);
+          const double e0 = __dsub_rn(xv, (double)p0[k]), e1 = __dsub_rn(xv, (double)p1[k]);
+          const double e2 = __dsub_rn(xv, (double)p2[k]), e3 = __dsub_rn(xv, (double)p3[k]);
+          d0 = __dadd_rn(d0, __dmul_rn(e0, e0));
+          d1 = __dadd_rn(d1, __dmul_rn(e1, e1));
+          d2 = __dadd_rn(d2, __dmul_rn(e2, e2));
+          d3 = __dadd_rn(d3, __dmul_rn(e3, e3));
+        }
+        if (d0 < best) { best = d0; bidx = c0; }
+        if (c1 < C && d1 < best) { best = d1; bidx = c1; }
+        if (c2 < C && d2 < best) { best = d2; bidx = c2; }
+        if (c3 < C && d3 < best) { best = d3; bidx = c3; }
       }
-    }
-  }
-}
-
-template <typename T, int D>
-__global__ void km_moves(const T* __restrict__ X, int64_t N, int C, const Move* __restrict__ moves,
-                         const unsigned long long* __restrict__ count, float* __restrict__ sums,
-                         int32_t* __restrict__ cnt) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t total = (int64_t)*count;
-  for (int64_t e = warp; e < total; e += nw) {
-    const Move mv = moves[e];
-    const int64_t h = mv.row / N;
-    const T* x = X + mv.row * D;
-    for (int k = lane * 4; k < D; k += 128) {
-      const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
-                                   Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
-      atomicAdd(reinterpret_cast<float4*>(sums + (h * C + mv.to) * D + k), v);
-      if (mv.from >= 0)
-        atomicAdd(reinterpret_cast<float4*>(sums + (h * C + mv.from) * D + k),
-                  make_float4(-v.x, -v.y, -v.z, -v.w));
-    }
-    if (lane == 0) {
-      atomicAdd(cnt + h * C + mv.to, 1);
-      if (mv.from >= 0) atomicAdd(cnt + h * C + mv.from, -1);
+      argmin_lanes(best, bidx, 32);
+      const int old = first ? -1 : labels[g];
+      __syncwarp();
+      if (lane == 0) labels[g] = bidx;
+      if (bidx != old) move_row<T, D>(x, sums, cnt, h * C + bidx, h * C + old, old >= 0, lane, 32);
     }
   }
 }
@@ -699,10 +685,9 @@ bool make_map_f16(CUtensorMap* map, const void* base, int64_t rows, int d, int b
 struct TcWs {
   float* sums;
   int32_t* cnt;
-  int64_t* refine_rows;
-  unsigned long long* counters;  // [0] full refine, [1] moves, [2] picks
-  Pick* picks;
-  Move* moves;
+  uint8_t* kind;
+  int4* cand;
+  int32_t* from;
   __half* xh;
   float* xnorm;
   __half* ch;
@@ -718,10 +703,9 @@ TcWs carve(Carver& cv, int64_t bh, int64_t n, int32_t d, int32_t c) {
   const int cp = c_pad_of(c);
   w.sums = cv.take<float>((size_t)bh * c * d);
   w.cnt = cv.take<int32_t>((size_t)bh * c);
-  w.refine_rows = cv.take<int64_t>((size_t)bh * n);
-  w.counters = cv.take<unsigned long long>(3);
-  w.picks = cv.take<Pick>((size_t)bh * n);
-  w.moves = cv.take<Move>((size_t)bh * n);
+  w.cand = cv.take<int4>((size_t)bh * n);
+  w.from = cv.take<int32_t>((size_t)bh * n);
+  w.kind = cv.take<uint8_t>((size_t)bh * n);
   w.xh = cv.take<__half>((size_t)bh * n * d);
   w.xnorm = cv.take<float>((size_t)bh * n);
   w.ch = cv.take<__half>((size_t)bh * cp * d);
@@ -742,6 +726,7 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   int* status = device_status_word();
   const int64_t rows = bh * n;
   const unsigned wgrid = (unsigned)std::min<int64_t>(ceil_div(rows, 8), 148 * 32);
+  const unsigned rgrid = (unsigned)std::min<int64_t>(ceil_div(ceil_div(rows, 32), 8), 148 * 32);
 
   if (cent != init)
     EAR_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * bh * c * D, cudaMemcpyDeviceToDevice, s));
@@ -765,12 +750,9 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   p.cmax = w.cmax;
   p.cbad = w.cbad;
   p.labels = labels;
-  p.refine_rows = w.refine_rows;
-  p.refine_count = w.counters;
-  p.moves = w.moves;
-  p.move_count = w.counters + 1;
-  p.picks = w.picks;
-  p.pick_count = w.counters + 2;
+  p.kind = w.kind;
+  p.cand = w.cand;
+  p.from = w.from;
   p.N = n;
   p.C = c;
   p.C_pad = cp;
@@ -787,16 +769,10 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   const int64_t crow = bh * (int64_t)c;
   for (int t = 0; t < iters; ++t) {
     p.first = t == 0 ? 1 : 0;
-    EAR_CUDA(cudaMemsetAsync(w.counters, 0, 3 * sizeof(unsigned long long), s));
     km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
     EAR_TRY(after_launch());
-    km_refine64<uint16_t, D><<<wgrid, 256, 0, s>>>(X, cent, n, c, labels, p.first, w.refine_rows,
-                                                   w.counters, w.sums, w.cnt);
-    EAR_TRY(after_launch());
-    km_pick64<uint16_t, D><<<wgrid, 256, 0, s>>>(X, cent, n, c, labels, p.first, w.picks,
-                                                 w.counters + 2, w.sums, w.cnt);
-    EAR_TRY(after_launch());
-    km_moves<uint16_t, D><<<wgrid, 256, 0, s>>>(X, n, c, w.moves, w.counters + 1, w.sums, w.cnt);
+    km_resolve<uint16_t, D><<<rgrid, 256, 0, s>>>(X, cent, n, c, rows, labels, p.first, w.kind,
+                                                  w.cand, w.from, w.sums, w.cnt);
     EAR_TRY(after_launch());
     EAR_CUDA(cudaMemsetAsync(w.cmax, 0, sizeof(float) * bh * 2, s));
     km_finalize<<<(unsigned)ceil_div(crow, 8), 256, 0, s>>>(w.sums, w.cnt, cent, counts, w.ch,

@@ -6,15 +6,19 @@
 // The second form is the one evaluated: each key is centred on its cluster
 // centroid once (one fp32 rounding per element) before the dot product, so
 // the small logit gaps are not the difference of two large fp32 logits.
-// Grid = (key cluster b, slice); a block walks its cluster's contiguous rows
-// in 64-row chunks against 64-centroid chunks of q̄ (4x4 register tiles).
+// Grid = (group of kClusters key clusters, slice).  A block holds the
+// slice's centroids q̄ transposed in shared memory ([k][a], up to 128 at a
+// time) and walks each cluster's contiguous rows in 64-row chunks, centred
+// and transposed ([k][j]); a thread accumulates an 8 x 4 tile (8 centroids x
+// 4 keys) from one 8-wide and one 4-wide vector load per k.
 #include "ear_internal.cuh"
 
 namespace ear {
 namespace {
 
-constexpr int kA = 64;     // query centroids per chunk
-constexpr int kJ = 64;     // keys per chunk
+constexpr int kA = 128;      // query centroids per pass
+constexpr int kJ = 64;       // keys per chunk
+constexpr int kClusters = 4; // key clusters per block
 constexpr int kThreads = 256;
 
 template <typename T, int D>
@@ -24,70 +28,104 @@ pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
          const int32_t* __restrict__ koff, int64_t Nk, int Cq, int Ck, float scale,
          float* __restrict__ E, int* status) {
   extern __shared__ float smem[];
-  float* qs = smem;                  // [kA][D + 1]
-  float* ks = smem + kA * (D + 1);   // [kJ][D + 1]
-  float* kbar = ks + kJ * (D + 1);   // [D]
+  float* qs = smem;               // [D][kA]
+  float* ks = qs + D * kA;        // [D][kJ]
+  float* kbar = ks + D * kJ;      // [D]
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int64_t h = blockIdx.y;
-  const int b = blockIdx.x;
   const int32_t* oh = koff + h * (int64_t)(Ck + 1);
-  int32_t r0 = oh[b], r1 = oh[b + 1];
-  if (r0 < 0 || r1 < r0 || r1 > Nk) {
-    if (tid == 0) latch(status, EAR_ERR_DEVICE);
-    r1 = r0 = 0;
-  }
   const T* kh = K + h * Nk * D;
-  for (int k = tid; k < D; k += kThreads) kbar[k] = kc[(h * Ck + b) * (int64_t)D + k];
 
   for (int a0 = 0; a0 < Cq; a0 += kA) {
     __syncthreads();
-    for (int e = tid; e < kA * D; e += kThreads) {
-      int r = e / D, k = e % D;
-      qs[r * (D + 1) + k] = (a0 + r) < Cq ? qc[(h * Cq + a0 + r) * (int64_t)D + k] : 0.f;
+    // q̄ chunk, transposed: lanes take consecutive centroids (conflict-free stores)
+    for (int e = tid; e < kA * (D / 4); e += kThreads) {
+      const int a = e % kA, k0 = (e / kA) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a0 + a < Cq) v = *reinterpret_cast<const float4*>(qc + (h * Cq + a0 + a) * (int64_t)D + k0);
+      qs[(k0 + 0) * kA + a] = v.x;
+      qs[(k0 + 1) * kA + a] = v.y;
+      qs[(k0 + 2) * kA + a] = v.z;
+      qs[(k0 + 3) * kA + a] = v.w;
     }
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j0 = r0; j0 < r1; j0 += kJ) {
-      const int nj = min(kJ, r1 - j0);
-      __syncthreads();
-      for (int e = tid; e < kJ * D; e += kThreads) {
-        int r = e / D, k = e % D;
-        ks[r * (D + 1) + k] = r < nj ? Elem<T>::load(kh, (int64_t)(j0 + r) * D + k) - kbar[k] : 0.f;
+    for (int bi = 0; bi < kClusters; ++bi) {
+      const int b = blockIdx.x * kClusters + bi;
+      if (b >= Ck) break;
+      int32_t r0 = oh[b], r1 = oh[b + 1];
+      if (r0 < 0 || r1 < r0 || r1 > Nk) {
+        if (tid == 0) latch(status, EAR_ERR_DEVICE);
+        r1 = r0 = 0;
       }
-      __syncthreads();
-      float acc[4][4];
+      __syncthreads();  // previous chunk's readers are done with ks / kbar
+      for (int k = tid; k < D; k += kThreads) kbar[k] = kc[(h * Ck + b) * (int64_t)D + k];
+      float part[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i) part[i] = 0.f;
+      for (int j0 = r0; j0 < r1; j0 += kJ) {
+        const int nj = min(kJ, r1 - j0);
+        __syncthreads();
+        // centred keys, transposed: lanes take consecutive rows
+        for (int e = tid; e < kJ * (D / 4); e += kThreads) {
+          const int j = e % kJ, k0 = (e / kJ) * 4;
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+          if (j < nj) {
+            const int64_t base = (int64_t)(j0 + j) * D + k0;
+            float x[4];
+            if constexpr (sizeof(T) == 2) {  // four bf16 in one 8-byte load
+              const uint2 w = *reinterpret_cast<const uint2*>(kh + base);
+              x[0] = __uint_as_float(w.x << 16);
+              x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+              x[2] = __uint_as_float(w.y << 16);
+              x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+            } else {
+              const float4 w = *reinterpret_cast<const float4*>(kh + base);
+              x[0] = w.x;
+              x[1] = w.y;
+              x[2] = w.z;
+              x[3] = w.w;
+            }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
-      for (int k = 0; k < D; ++k) {
-        float qv[4], kv[4];
+            for (int i = 0; i < 4; ++i) v[i] = x[i] - kbar[k0 + i];
+          }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) qv[i] = qs[(ty + 16 * i) * (D + 1) + k];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) kv[j] = ks[(tx + 16 * j) * (D + 1) + k];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float g = scale * acc[i][j];  // zero for padded rows (centred value 0)
-          part[i] = fmaf(g, g, part[i]);
+          for (int i = 0; i < 4; ++i) ks[(k0 + i) * kJ + j] = v[i];
         }
-    }
+        __syncthreads();
+        float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float v = part[i];
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      const int a = a0 + ty + 16 * i;
-      if (tx == 0 && a < Cq) {
-        const bool live = qn[h * Cq + a] > 0 && r1 > r0;
-        E[(h * Cq + a) * (int64_t)Ck + b] = live ? v : 0.f;
+          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < D; ++k) {
+          const float4 q0 = *reinterpret_cast<const float4*>(qs + k * kA + ty * 8);
+          const float4 q1 = *reinterpret_cast<const float4*>(qs + k * kA + ty * 8 + 4);
+          const float4 kv = *reinterpret_cast<const float4*>(ks + k * kJ + tx * 4);
+          const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kk[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float g = scale * acc[i][j];  // zero for padded rows (centred value 0)
+            part[i] = fmaf(g, g, part[i]);
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float v = part[i];
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        const int a = a0 + ty * 8 + i;
+        if (tx == 0 && a < Cq) {
+          const bool live = qn[h * Cq + a] > 0 && r1 > r0;
+          E[(h * Cq + a) * (int64_t)Ck + b] = live ? v : 0.f;
+        }
       }
     }
   }
@@ -97,10 +135,10 @@ template <typename T, int D>
 ear_status run_t(const float* qc, const int32_t* qn, const float* kc, const void* K,
                  const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q, int32_t c_k,
                  float scale, float* E, cudaStream_t s) {
-  const size_t smem = ((size_t)(kA + kJ) * (D + 1) + D) * sizeof(float);
+  const size_t smem = ((size_t)(kA + kJ) * D + D) * sizeof(float);
   EAR_CUDA(cudaFuncSetAttribute(pr_probe<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem));
-  pr_probe<T, D><<<dim3((unsigned)c_k, (unsigned)bh), kThreads, smem, s>>>(
+  pr_probe<T, D><<<dim3((unsigned)ceil_div(c_k, kClusters), (unsigned)bh), kThreads, smem, s>>>(
       qc, qn, kc, (const T*)K, koff, n_k, c_q, c_k, scale, E, device_status_word());
   return after_launch();
 }

@@ -12,8 +12,11 @@
 // digit at which the running cost crosses the remaining budget.  Ratios are
 // correctly rounded fp64 divisions, so the order matches a host fp64 sort.
 //
-// One 1024-thread block per slice: select, mark, count per query cluster,
-// scan, and emit each query cluster's exact key clusters in ascending order.
+// One 1024-thread block per slice: keys and costs once into the workspace,
+// select (each pass: a warp whose lanes share one digit adds the costs in
+// registers and makes one shared-memory atomic; warp 0 scans the histogram),
+// mark, count per query cluster, scan, and emit each query cluster's exact
+// key clusters in ascending order.
 #include "ear_internal.cuh"
 
 namespace ear {
@@ -64,7 +67,8 @@ __global__ void __launch_bounds__(kThreads)
 rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
          const int32_t* __restrict__ kn_all, int Cq, int Ck, int64_t budget, int mode,
          uint8_t* __restrict__ exact_all, int32_t* __restrict__ blk_off_all,
-         int32_t* __restrict__ blk_list_all, int64_t* __restrict__ pairs) {
+         int32_t* __restrict__ blk_list_all, int64_t* __restrict__ pairs,
+         uint64_t* __restrict__ khi_ws, unsigned long long* __restrict__ cost_ws) {
   __shared__ unsigned long long hist[256];
   __shared__ uint64_t s_phi;
   __shared__ uint32_t s_plo;
@@ -83,6 +87,8 @@ rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
   uint8_t* exact = exact_all + h * (int64_t)nblk;
   int32_t* blk_off = blk_off_all + h * (int64_t)(Cq + 1);
   int32_t* blk_list = blk_list_all + h * (int64_t)nblk;
+  uint64_t* khi = khi_ws + h * (int64_t)nblk;
+  unsigned long long* cost = cost_ws + h * (int64_t)nblk;
 
   if (tid == 0) {
     s_phi = 0;
@@ -91,34 +97,79 @@ rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
     s_all_fit = 0;
     s_total = 0;
   }
+  // keys once (cost 0 = never exact)
+  for (int idx = tid; idx < nblk; idx += kThreads) {
+    Key k;
+    unsigned long long c = 0;
+    if (!block_key(Eh, qn, kn, Ck, mode, idx, k, c)) {
+      k.hi = 0;
+      c = 0;
+    }
+    khi[idx] = k.hi;
+    cost[idx] = c;
+  }
   for (int pass = 0; pass < 12; ++pass) {
     for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
     __syncthreads();
     const uint64_t phi = s_phi;
     const uint32_t plo = s_plo;
-    for (int idx = tid; idx < nblk; idx += kThreads) {
+    for (int base = 0; base < nblk; base += kThreads) {
+      const int idx = base + tid;
       Key k;
-      unsigned long long c;
-      if (!block_key(Eh, qn, kn, Ck, mode, idx, k, c)) continue;
-      if (!prefix_match(k, pass, phi, plo)) continue;
-      atomicAdd(&hist[digit_of(k, pass)], c);
+      unsigned long long c = 0;
+      if (idx < nblk) {
+        k.hi = khi[idx];
+        k.lo = (uint32_t)idx;
+        c = cost[idx];
+      }
+      const bool want = c > 0 && prefix_match(k, pass, phi, plo);
+      const int d = want ? digit_of(k, pass) : -1;
+      // the early passes see one digit across the warp: add in registers
+      if (__all_sync(0xffffffffu, d == __shfl_sync(0xffffffffu, d, 0) && want)) {
+        unsigned long long sum = c;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0) atomicAdd(&hist[d], sum);
+      } else if (want) {
+        atomicAdd(&hist[d], c);
+      }
     }
     __syncthreads();
-    if (tid == 0) {
+    if (wid == 0) {
+      // first digit u with (costs below u) + hist[u] > remaining budget
       const unsigned long long rem = (unsigned long long)s_rem;
-      unsigned long long cum = 0;
-      int t = -1;
-      for (int u = 0; u < 256; ++u) {
-        if (cum + hist[u] > rem) {
-          t = u;
-          break;
-        }
-        cum += hist[u];
+      unsigned long long v[8], loc = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = hist[lane * 8 + i];
+        loc += v[i];
       }
-      if (t < 0) {
-        s_all_fit = 1;  // everything fits: only possible in the first pass
-        if (pass == 0) s_total = cum;
-      } else {
+      unsigned long long incl = loc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const unsigned long long excl = incl - loc;
+      const bool mine = excl <= rem && incl > rem;
+      const unsigned m = __ballot_sync(0xffffffffu, mine);
+      const unsigned long long total = __shfl_sync(0xffffffffu, incl, 31);
+      if (m == 0) {
+        if (lane == 0) {
+          s_all_fit = 1;  // everything fits: only possible in the first pass
+          if (pass == 0) s_total = total;
+        }
+      } else if (mine) {
+        unsigned long long cum = excl;
+        int t = lane * 8 + 7;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (cum + v[i] > rem) {
+            t = lane * 8 + i;
+            break;
+          }
+          cum += v[i];
+        }
         s_rem = (long long)(rem - cum);
         if (pass < 8)
           s_phi |= (uint64_t)t << (56 - 8 * pass);
@@ -130,14 +181,15 @@ rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
     if (s_all_fit) break;
   }
   const bool all_fit = s_all_fit != 0;
-  const uint64_t khi = s_phi;
-  const uint32_t klo = s_plo;
+  const uint64_t kstar_hi = s_phi;
+  const uint32_t kstar_lo = s_plo;
 
   // mark
   for (int idx = tid; idx < nblk; idx += kThreads) {
     Key k;
-    unsigned long long c;
-    bool ex = block_key(Eh, qn, kn, Ck, mode, idx, k, c) && (all_fit || key_less(k, khi, klo));
+    k.hi = khi[idx];
+    k.lo = (uint32_t)idx;
+    const bool ex = cost[idx] > 0 && (all_fit || key_less(k, kstar_hi, kstar_lo));
     exact[idx] = ex ? 1 : 0;
   }
   if (tid == 0) pairs[h] = all_fit ? (int64_t)s_total : (int64_t)(budget - s_rem);
@@ -196,14 +248,19 @@ rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
 
 }  // namespace
 
-size_t route_workspace(int64_t, int32_t, int32_t) { return 0; }
+// keys (fp64 ratio bits) and costs of every block, 8 + 8 bytes each
+size_t route_workspace(int64_t bh, int32_t c_q, int32_t c_k) {
+  return (size_t)bh * c_q * c_k * 16;
+}
 
 ear_status route_run(const float* E, const int32_t* qn, const int32_t* kn, int64_t bh,
                      int64_t budget, int32_t c_q, int32_t c_k, int32_t mode, uint8_t* exact,
-                     int32_t* blk_off, int32_t* blk_list, int64_t* pairs, void*,
+                     int32_t* blk_off, int32_t* blk_list, int64_t* pairs, void* ws,
                      cudaStream_t s) {
+  uint64_t* khi = static_cast<uint64_t*>(ws);
+  unsigned long long* cost = reinterpret_cast<unsigned long long*>(khi + bh * c_q * c_k);
   rt_route<<<(unsigned)bh, kThreads, 0, s>>>(E, qn, kn, c_q, c_k, budget, mode, exact, blk_off,
-                                             blk_list, pairs);
+                                             blk_list, pairs, khi, cost);
   return after_launch();
 }
 
