@@ -192,6 +192,25 @@ def run_reference(args, w):
     return 0
 
 
+def recorded_traffic(heads: int):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, scaled to `heads`, or None when the kernel source has changed
+    since the capture (the counters no longer describe it)."""
+    import hashlib
+
+    here = os.path.dirname(os.path.abspath(__file__))
+    prof = os.path.join(here, "profiles", "attention_tc_wan.md")
+    src = os.path.join(here, "clustered_block_sparse_b200", "csrc", "attention_tc.cu")
+    try:
+        text = open(prof).read()
+        per_head = int(text.split("traffic_bytes_per_head:")[1].split()[0])
+        sha = text.split("kernel_source_sha256:")[1].split()[0]
+        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except (OSError, IndexError, ValueError):
+        return None
+    return per_head * heads if sha == cur else None
+
+
 def config_of(w, n_gpus):
     return {"workload": w.name, "heads": w.heads, "n_q": w.n, "n_k": w.n, "d": w.d,
             "c_q": w.c_q, "c_k": w.c_k, "kmeans_iters": w.iters, "density": w.density,
@@ -206,7 +225,7 @@ def run_ear(args, w):
     import torch.distributed as dist
 
     from clustered_block_sparse_b200 import _native as nat
-    from clustered_block_sparse_b200 import ear
+    from clustered_block_sparse_b200 import ear, replicas
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -222,13 +241,9 @@ def run_ear(args, w):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if not distributed:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, device=torch.device("cuda", local))
 
-    heads = list(range(rank * w.heads, (rank + 1) * w.heads))
+    heads = replicas.rank_heads(rank, w.heads)
     layer = gen.make_layer(w, heads=heads)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     dev = torch.device("cuda", local)
@@ -315,7 +330,7 @@ def run_ear(args, w):
 
     line = {
         "metric": METRIC,
-        "value": ms_step / world,
+        "value": replicas.job_ms_per_layer(ms_step, world),
         "unit": "ms/layer",
         "n_gpus": world,
         "steps": args.steps,
@@ -337,7 +352,10 @@ def run_ear(args, w):
         "roofline": {"bound": "tensor", "kernel": "ear_attention", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
-                     "traffic": None,
+                     "traffic": recorded_traffic(w.heads),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                       "at_tc at 4 heads (profiles/attention_tc_wan.md), "
+                                       "scaled by heads; null if the kernel changed since",
                      "algorithmic_bytes": attention_bytes(w),
                      "algorithmic_flops": fl["attention"]},
         "e2e": e2e,
@@ -393,6 +411,79 @@ def time_e2e(args, w, layer, ear, dev, tdt, stream):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+def run_skew_study(args):
+    """Skewed cluster sizes (Zipf 1.2 mixture, Wan shape, heads 0 and 1): the
+    relative L2 error against dense attention, on 4096 seeded query rows per
+    head, of (i) error-routed attention with compensation (the method), (ii)
+    routing by the centroid block mass P_ab = |b| e^(s q̄_a·k̄_b) / sum over b'
+    with compensation, (iii) the same routing with the skipped blocks dropped,
+    at each density.  All three use the same global prefix budget; the score
+    key enters ear_route as E = P_ab |b|, so its E/|b| ratio is P_ab.  The
+    dense reference and the score key are plain fp64 torch on the GPU
+    (measurement only); every routed output comes from the library."""
+    import torch
+
+    from clustered_block_sparse_b200 import ear
+
+    w = gen.SKEW
+    heads = [0, 1]
+    layer = gen.make_layer(w, heads=heads)
+    dev = torch.device("cuda", 0)
+    tdt = torch.bfloat16
+    q = torch.from_numpy(layer.q).to(dev, tdt)
+    k = torch.from_numpy(layer.k).to(dev, tdt)
+    v = torch.from_numpy(layer.v).to(dev, tdt)
+    qi = torch.from_numpy(layer.q_init).to(dev)
+    ki = torch.from_numpy(layer.k_init).to(dev)
+    s = 1.0 / math.sqrt(w.d)
+    qc, ql, qn = ear.ear_kmeans(q, qi, w.iters)
+    kc, kl, kn = ear.ear_kmeans(k, ki, w.iters)
+    qp, qo, qx, _ = ear.ear_permute(ql, w.c_q, q)
+    kp, ko, kx, _ = ear.ear_permute(kl, w.c_k, k)
+    _, _, vx, vm = ear.ear_permute(kl, w.c_k, v, seg_mean=True)
+    e_err = ear.ear_probe(qc, qn, kc, kx, ko)
+    knd = kn.double()
+    logw = s * torch.einsum("had,hbd->hab", qc.double(), kc.double()) + torch.log(knd).unsqueeze(1)
+    e_score = (torch.softmax(logw, dim=2) * knd.unsqueeze(1)).float().contiguous()
+
+    rng = np.random.default_rng(5005)
+    n_rows = 4096
+    rows = [torch.from_numpy(np.sort(rng.choice(w.n, n_rows, replace=False))).to(dev)
+            for _ in heads]
+    dense = []
+    for h in range(len(heads)):
+        kh, vh = k[h].double(), v[h].double()
+        parts = []
+        for c0 in range(0, n_rows, 512):
+            qs = q[h, rows[h][c0:c0 + 512]].double()
+            parts.append(torch.softmax(s * qs @ kh.T, dim=1) @ vh)
+        dense.append(torch.cat(parts))
+    ref_norm = math.sqrt(sum(float((d_ ** 2).sum()) for d_ in dense))
+
+    variants = (("error_routed_compensated", e_err, True),
+                ("score_routed_compensated", e_score, True),
+                ("score_routed_dropped", e_score, False))
+    table = {}
+    for rho in gen.SKEW_DENSITIES:
+        row = {}
+        for name, e, comp in variants:
+            exact, bo, bl, pairs = ear.ear_route(e, qn, kn, w.n, w.n, rho)
+            o, _ = ear.ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl,
+                                     compensate=comp)
+            err2 = sum(float(((o[h, rows[h]].double() - dense[h]) ** 2).sum())
+                       for h in range(len(heads)))
+            row[name] = math.sqrt(err2) / ref_norm
+        row["exact_pair_fraction"] = float(pairs.double().sum()) / (len(heads) * w.n * w.n)
+        table[f"{rho:.2f}"] = row
+    if ear.ear_get_device_status() != 0:
+        raise RuntimeError("device status latched an error in the study")
+    print(json.dumps({"study": "skew", "workload": w.name, "heads": heads,
+                      "sampled_query_rows_per_head": n_rows, "metric": "relative L2 vs dense",
+                      "dense_reference": "fp64 softmax(s q K^T) V on the sampled rows",
+                      "rel_l2": table}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -404,7 +495,11 @@ def main(argv=None):
                     help="override the head count (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--study", choices=("skew",), default=None,
+                    help="run a quality study instead of the timing line")
     args = ap.parse_args(argv)
+    if args.study == "skew":
+        return run_skew_study(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]

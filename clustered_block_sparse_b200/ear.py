@@ -175,6 +175,13 @@ def ear_attention(q_perm_x, k_perm_x, v_perm_x, q_offsets, k_offsets, q_perm, k_
     return o, lse
 
 
+def ear_selftest_wait_timeout(device=None) -> None:
+    """Enqueue the bounded-wait self-test: the next ear_get_device_status() on
+    this device reports EAR_ERR_TIMEOUT (after about one second)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    N.check("ear_selftest_wait_timeout", N.lib().ear_selftest_wait_timeout(_stream(dev)))
+
+
 def ear_get_device_status(device=None) -> int:
     """Synchronize the current stream and return (and clear) the latched device status."""
     dev = torch.device("cuda") if device is None else torch.device(device)

@@ -242,6 +242,17 @@ EAR_API ear_status ear_get_device_status(int32_t* out, void* stream);
 /* Number of kernels this library has launched in this process (all devices). */
 EAR_API uint64_t ear_launch_count(void);
 
+/*
+ * Failure-path self-test (the pages have no counterpart; it checks this
+ * library's bounded waits).  Enqueues one warp on `stream` that waits on a
+ * barrier nothing completes.  The wait gives up after its bound (about 1 s),
+ * latches EAR_ERR_TIMEOUT in the device status word and the kernel returns;
+ * the next ear_get_device_status() on this device reports EAR_ERR_TIMEOUT and
+ * clears it, and the context stays usable.  Returns EAR_ERR_CUDA if the launch
+ * fails; takes no buffers and allocates nothing.
+ */
+EAR_API ear_status ear_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif
