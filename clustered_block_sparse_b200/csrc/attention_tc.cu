@@ -4,7 +4,7 @@
 //
 // One CTA = one unit of up to 256 permuted query rows of ONE query cluster a,
 // split in two 128-row tiles A and B (tcgen05.mma M = 128).  Both tiles walk
-// the same key chunks.  A chunk is up to four 32-row boxes (128 keys):
+// the same key chunks.  A chunk is up to two 32-row boxes (64 keys):
 //   * exact boxes: the rows of every key cluster b listed for a, 32 at a
 //     time (the last box of a cluster is partial), so small clusters share
 //     a chunk instead of each paying for a whole MMA round;
@@ -13,22 +13,23 @@
 //     clusters that are exact for a or empty.  Exact and centroid boxes never
 //     share a chunk.
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then chunk boxes into a 2-stage
+//   warp 0      TMA producer: Q tiles once, then chunk boxes into a 4-stage
 //               ring.  It publishes each stage's chunk descriptor (box count,
 //               valid rows per box, centroid or not, bias) in shared memory
 //               and ends the sequence with an empty descriptor.
-//   warp 1      MMA issuer (one elected lane of the warp): S_t = Q_t K^T into TMEM, then
-//               O_t += P_t V with P_t read from TMEM.  Issue order
-//               QK_A(c) QK_B(c) | PV_A(c) QK_A(c+1) PV_B(c) QK_B(c+1) | ...
-//               so one tile's softmax overlaps the other tile's MMAs.
+//   warp 1      MMA issuer (one elected lane of the warp): S_t = Q_t K^T into
+//               one of two TMEM buffers per tile, then O_t += P_t V with P_t
+//               read from TMEM.  Issue order
+//               QK_A(0) QK_B(0) QK_A(1) QK_B(1) | PV_A(c) QK_A(c+2) PV_B(c) QK_B(c+2) | ...
+//               so the next chunk's scores are ready while the softmax works.
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread
 //               per query row (= TMEM lane).  Online softmax in base 2 on the
 //               raw scores: an exact chunk is read from TMEM once (max, then
 //               exponent, from registers); the exponent argument is one packed
 //               FMA per score pair; the running max only moves (and O is
 //               rescaled in TMEM) when it grows by more than 2^8.
-// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512);
-// P_t (bf16 pairs) overwrites the first half of S_t.
+// TMEM (512 columns): S_A0 [0,64), S_A1 [64,128), S_B0 [128,192), S_B1 [192,256),
+// O_A [256,384), O_B [384,512); P (bf16 pairs) overwrites the first half of its S buffer.
 #include <mutex>
 
 #include "ear_internal.cuh"
@@ -43,9 +44,11 @@ constexpr int kTileRows = 128;
 constexpr int kTiles = 2;
 constexpr int kUnitRows = kTileRows * kTiles;
 constexpr int kBox = 32;                 // rows per TMA box
-constexpr int kBoxes = 4;                // boxes per chunk
-constexpr int kChunk = kBox * kBoxes;    // keys per chunk (MMA N <= 128)
-constexpr int kStages = 2;
+constexpr int kBoxes = 2;                // boxes per chunk
+constexpr int kChunk = kBox * kBoxes;    // keys per chunk
+constexpr int kStages = 4;               // K/V ring depth (chunks)
+constexpr int kSBufs = 2;                // S buffers per tile: Q K^T of chunk c+1 runs
+                                         // while the softmax works on chunk c
 constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -61,14 +64,17 @@ constexpr int kRegsLaunch = 168;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 // barrier slots
-constexpr int kBarKvFull = 0;   // + stage
-constexpr int kBarKvEmpty = 2;  // + stage
-constexpr int kBarQFull = 4;
-constexpr int kBarSFull = 5;    // + tile
-constexpr int kBarPFull = 7;    // + tile
-constexpr int kBarODone = 9;    // + tile
-constexpr int kBarDrain = 11;   // teardown: every MMA issued has finished
-constexpr int kNumBars = 12;
+constexpr int kBarKvFull = 0;                     // + stage
+constexpr int kBarKvEmpty = kStages;              // + stage
+constexpr int kBarQFull = 2 * kStages;
+constexpr int kBarSFull = kBarQFull + 1;          // + tile * kSBufs + buffer
+constexpr int kBarPFull = kBarSFull + kTiles * kSBufs;  // + tile * kSBufs + buffer
+// O_t += P V of chunk c done: one barrier per (tile, S buffer of c).  With two
+// S buffers a softmax warp at chunk c only knows that P V of chunk c-2 has
+// finished; per-buffer barriers keep every parity wait within one phase.
+constexpr int kBarODone = kBarPFull + kTiles * kSBufs;  // + tile * kSBufs + buffer
+constexpr int kBarDrain = kBarODone + kTiles * kSBufs;  // teardown: every MMA issued has finished
+constexpr int kNumBars = kBarDrain + 1;
 
 // Chunk descriptor published by the producer for each stage.
 struct ChunkInfo {
@@ -79,12 +85,14 @@ struct ChunkInfo {
 
 template <int D>
 struct Layout {
-  static constexpr int kHalfBytes = kTileRows * 128;  // 128 rows x 64 bf16
+  static constexpr int kHalfBytes = kTileRows * 128;  // Q tile: 128 rows x 64 bf16 per half
   static constexpr int kTileBytes = kHalfBytes * (D / 64);
+  static constexpr int kSHalf = kChunk * 128;         // K / V stage: 64 rows x 64 bf16 per half
+  static constexpr int kStageBytes = kSHalf * (D / 64);
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTiles * kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBias = kV + kStages * kTileBytes;       // [stage][128] float
+  static constexpr int kV = kK + kStages * kStageBytes;
+  static constexpr int kBias = kV + kStages * kStageBytes;      // [stage][kChunk] float
   static constexpr int kInfo = kBias + kStages * kChunk * 4;    // [stage] ChunkInfo
   static constexpr int kList = kInfo + kStages * 32;              // unit's exact key clusters
   static constexpr int kKoff = kList + kTableMax * 4;             // slice's key offsets
@@ -305,21 +313,19 @@ __device__ __forceinline__ void producer_role(
     // The next chunk: up to four boxes of the same kind, held in registers
     // (static indices).  It is gathered while the ring slot is still busy.
     int comp = 0, nbox = 0;
-    int32_t r0 = 0, r1 = 0, r2 = 0, r3 = 0, comp_first = 0;
-    int v0 = 0, v1 = 0, v2 = 0, v3 = 0;
+    int32_t r0 = 0, r1 = 0, comp_first = 0;
+    int v0 = 0, v1 = 0;
     auto gather = [&]() {
       comp = have && bcomp ? 1 : 0;
       nbox = 0;
-      r0 = r1 = r2 = r3 = 0;
-      v0 = v1 = v2 = v3 = 0;
+      r0 = r1 = 0;
+      v0 = v1 = 0;
       comp_first = brow;
 #pragma unroll
       for (int k = 0; k < kBoxes; ++k) {
         if (!(have && (bcomp ? 1 : 0) == comp)) break;
         if (k == 0) { r0 = brow; v0 = bval; }
         if (k == 1) { r1 = brow; v1 = bval; }
-        if (k == 2) { r2 = brow; v2 = bval; }
-        if (k == 3) { r3 = brow; v3 = bval; }
         nbox = k + 1;
         have = it.next(brow, bval, bcomp);
       }
@@ -335,7 +341,7 @@ __device__ __forceinline__ void producer_role(
         for (int j = lane; j < kChunk; j += 32) {
           float bv = -INFINITY;
           const int bx = j / kBox;
-          const int vb = bx == 0 ? v0 : bx == 1 ? v1 : bx == 2 ? v2 : v3;
+          const int vb = bx == 0 ? v0 : v1;
           if (bx < nbox && (j % kBox) < vb) {
             const int b = comp_first + j;
             const int32_t cnt = koff_t[b + 1] - koff_t[b];
@@ -351,8 +357,6 @@ __device__ __forceinline__ void producer_role(
         ci->comp = comp;
         ci->valid[0] = v0;
         ci->valid[1] = v1;
-        ci->valid[2] = v2;
-        ci->valid[3] = v3;
         if (nbox == 0)
           mbar_arrive(&bars[kBarKvFull + s]);  // end of the sequence
         else
@@ -362,17 +366,17 @@ __device__ __forceinline__ void producer_role(
         const CUtensorMap* mk = comp ? &tmKc : &tmK;
         const CUtensorMap* mv = comp ? &tmVc : &tmV;
         const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
-        uint8_t* kdst = smem + L::kK + s * L::kTileBytes;
-        uint8_t* vdst = smem + L::kV + s * L::kTileBytes;
+        uint8_t* kdst = smem + L::kK + s * L::kStageBytes;
+        uint8_t* vdst = smem + L::kV + s * L::kStageBytes;
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
-          const int32_t rw = bx == 0 ? r0 : bx == 1 ? r1 : bx == 2 ? r2 : r3;
+          const int32_t rw = bx == 0 ? r0 : r1;
 #pragma unroll
           for (int hf = 0; hf < D / 64; ++hf) {
             if (bx < nbox && leader) {
-              tma_load_2d(kdst + hf * L::kHalfBytes + bx * kBox * 128, mk, &bars[kBarKvFull + s],
+              tma_load_2d(kdst + hf * L::kSHalf + bx * kBox * 128, mk, &bars[kBarKvFull + s],
                           64 * hf, base + rw);
-              tma_load_2d(vdst + hf * L::kHalfBytes + bx * kBox * 128, mv, &bars[kBarKvFull + s],
+              tma_load_2d(vdst + hf * L::kSHalf + bx * kBox * 128, mv, &bars[kBarKvFull + s],
                           64 * hf, base + rw);
             }
           }
@@ -403,25 +407,26 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
       // warp-uniform); one elected lane issues the MMAs and commits.
       const bool leader = elect_one();
       const uint32_t idesc_pv = idesc_bf16(128, D, true);
-      auto issue_qk = [&](int t, int s, int n) {
+      // S of tile t, buffer b: TMEM columns [128 t + 64 b, +64); O_t: [256 + 128 t, +128)
+      auto issue_qk = [&](int t, int buf, int s, int n) {
         const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
-        const uint32_t qb = smem_u32(smem + L::kQ + t * L::kTileBytes);
-        const uint32_t kb = smem_u32(smem + L::kK + s * L::kTileBytes);
-        const uint64_t qd = desc_sw128(qb, 16, 1024), kd = desc_sw128(kb, 16, 1024);
+        const uint64_t qd = desc_sw128(smem_u32(smem + L::kQ + t * L::kTileBytes), 16, 1024);
+        const uint64_t kd = desc_sw128(smem_u32(smem + L::kK + s * L::kStageBytes), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * L::kHalfBytes + (kk % 4) * 32) >> 4;
-          if (leader) mma_ss(tmem + kTileRows * t, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+          const uint32_t qo = ((kk / 4) * L::kHalfBytes + (kk % 4) * 32) >> 4;
+          const uint32_t ko = ((kk / 4) * L::kSHalf + (kk % 4) * 32) >> 4;
+          if (leader)
+            mma_ss(tmem + kTileRows * t + kChunk * buf, qd + qo, kd + ko, idesc, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, int n, bool first) {
-        const uint32_t vb = smem_u32(smem + L::kV + s * L::kTileBytes);
-        const uint64_t vd = desc_sw128(vb, L::kHalfBytes, 1024);
+      auto issue_pv = [&](int t, int buf, int s, int n, bool first) {
+        const uint64_t vd = desc_sw128(smem_u32(smem + L::kV + s * L::kStageBytes), L::kSHalf, 1024);
         const int nk = n / 16;
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
           if (kk < nk && leader)
-            mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kk * 8,
+            mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kChunk * buf + kk * 8,
                    vd + ((kk * 2048) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
       };
@@ -429,39 +434,50 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
         if (leader) mma_commit(bar);
         __syncwarp();
       };
+      // n0, n1: keys of chunks c and c+1 (0 = past the end)
       bool ok = mbar_wait_warp(&bars[kBarQFull], 0, abort) &&
                 mbar_wait_warp(&bars[kBarKvFull], 0, abort);
-      int n_cur = ok ? info[0].nbox * kBox : 0;
-      if (ok && n_cur > 0) {
+      int n0 = ok ? info[0].nbox * kBox : 0, n1 = 0;
+      if (ok && n0 > 0) {
         tc_fence_after();
         for (int t = 0; t < ntiles; ++t) {
-          issue_qk(t, 0, n_cur);
-          commit(&bars[kBarSFull + t]);
+          issue_qk(t, 0, 0, n0);
+          commit(&bars[kBarSFull + t * kSBufs]);
+        }
+        ok = mbar_wait_warp(&bars[kBarKvFull + 1], 0, abort);
+        n1 = ok ? info[1].nbox * kBox : 0;
+        if (ok && n1 > 0) {
+          tc_fence_after();
+          for (int t = 0; t < ntiles; ++t) {
+            issue_qk(t, 1, 1, n1);
+            commit(&bars[kBarSFull + t * kSBufs + 1]);
+          }
         }
       }
-      for (int c = 0; ok && n_cur > 0; ++c) {
-        const int s = c % kStages;
-        const int s2 = (c + 1) % kStages;
-        int n_nxt = 0;
+      for (int c = 0; ok && n0 > 0; ++c) {
+        const int s = c % kStages, buf = c & 1;
+        const int s2 = (c + 2) % kStages;
+        int n2 = 0;
         for (int t = 0; t < ntiles && ok; ++t) {
-          ok = mbar_wait_warp(&bars[kBarPFull + t], c & 1, abort);
+          ok = mbar_wait_warp(&bars[kBarPFull + t * kSBufs + buf], (c >> 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, s, n_cur, c == 0);
-          commit(&bars[kBarODone + t]);
+          issue_pv(t, buf, s, n0, c == 0);
+          commit(&bars[kBarODone + t * kSBufs + buf]);
           if (t == ntiles - 1) commit(&bars[kBarKvEmpty + s]);
-          if (t == 0) {
-            ok = mbar_wait_warp(&bars[kBarKvFull + s2], ((c + 1) / kStages) & 1, abort);
+          if (t == 0 && n1 > 0) {
+            ok = mbar_wait_warp(&bars[kBarKvFull + s2], ((c + 2) / kStages) & 1, abort);
             if (!ok) break;
-            n_nxt = info[s2].nbox * kBox;
+            n2 = info[s2].nbox * kBox;
             tc_fence_after();
           }
-          if (n_nxt > 0) {
-            issue_qk(t, s2, n_nxt);
-            commit(&bars[kBarSFull + t]);
+          if (n2 > 0) {  // chunk c+2 into the buffer P V of chunk c has just read
+            issue_qk(t, buf, s2, n2);
+            commit(&bars[kBarSFull + t * kSBufs + buf]);
           }
         }
-        n_cur = n_nxt;
+        n0 = n1;
+        n1 = n2;
       }
       // every MMA issued above has finished before TMEM is released
       commit(&bars[kBarDrain]);
@@ -485,7 +501,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
     const int rows_t = t == 0 ? rows_a : rows_b;
     if (t < ntiles) {
       const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_bits + kTileRows * t;
+      const uint32_t tS0 = tmem + lane_bits + kTileRows * t;  // S buffer 0 of this tile
       const uint32_t tO = tmem + lane_bits + 256 + kTileRows * t;
       const float scale = p.qk_scale;
       const unsigned long long scale2 = pack2(__float_as_uint(scale), __float_as_uint(scale));
@@ -501,24 +517,23 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
         const int nbox = ci->nbox;
         const bool comp = ci->comp != 0;
         if (nbox == 0) break;
-        ok = mbar_wait_warp(&bars[kBarSFull + t], c & 1, abort);
+        const int buf = c & 1;
+        const uint32_t tS = tS0 + kChunk * buf;
+        ok = mbar_wait_warp(&bars[kBarSFull + t * kSBufs + buf], (c >> 1) & 1, abort);
         if (!ok) break;
         tc_fence_after();
         const float* bs = bias + s * kChunk;
         bool resc = false;
         float corr = 1.f, m_use = m;
         if (!comp) {
-          // exact chunk: one TMEM trip for all four boxes (unused boxes have
+          // exact chunk: one TMEM trip for both boxes (an unused box has
           // valid = 0), max and exponent from registers
-          const int v0 = ci->valid[0], v1 = ci->valid[1], v2 = ci->valid[2], v3 = ci->valid[3];
-          uint32_t x0[32], x1[32], x2[32], x3[32];
+          const int v0 = ci->valid[0], v1 = ci->valid[1];
+          uint32_t x0[32], x1[32];
           tmem_ld32(tS, x0);
           tmem_ld32(tS + 32, x1);
-          tmem_ld32(tS + 64, x2);
-          tmem_ld32(tS + 96, x3);
           tmem_ld_wait();
-          const float mx = fmaxf(fmaxf(box_max_raw(x0, v0), box_max_raw(x1, v1)),
-                                 fmaxf(box_max_raw(x2, v2), box_max_raw(x3, v3))) * scale;
+          const float mx = fmaxf(box_max_raw(x0, v0), box_max_raw(x1, v1)) * scale;
           if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
             if (m != -INFINITY) {
               resc = true;
@@ -536,14 +551,6 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
           if (nbox > 1) {
             lsum = add2(lsum, box_exp_c(x1, n2, scale2, none ? 0 : v1, pk));
             tmem_st16(tS + 16, pk);
-          }
-          if (nbox > 2) {
-            lsum = add2(lsum, box_exp_c(x2, n2, scale2, none ? 0 : v2, pk));
-            tmem_st16(tS + 32, pk);
-          }
-          if (nbox > 3) {
-            lsum = add2(lsum, box_exp_c(x3, n2, scale2, none ? 0 : v3, pk));
-            tmem_st16(tS + 48, pk);
           }
         } else {
           // centroid chunk, pass 1: chunk max (scaled, with the bias)
@@ -585,7 +592,9 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
         }
         tmem_st_wait();
         if (__any_sync(0xffffffffu, resc)) {
-          ok = mbar_wait_warp(&bars[kBarODone + t], (c - 1) & 1, abort);
+          // P V of chunk c-1 (c-2 and earlier are done: S of chunk c was written after them)
+          ok = mbar_wait_warp(&bars[kBarODone + t * kSBufs + ((c - 1) & 1)], ((c - 1) >> 1) & 1,
+                              abort);
           if (!ok) break;
           tc_fence_after();
           for (int g = 0; g < D / 32; ++g) {
@@ -600,7 +609,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
         }
         m = m_use;
         tc_fence_before();
-        mbar_arrive(&bars[kBarPFull + t]);
+        mbar_arrive(&bars[kBarPFull + t * kSBufs + buf]);
       }
       // epilogue: O / l written at the queries' original positions
       const float l = lo_f(lsum) + hi_f(lsum);
@@ -608,7 +617,13 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
       const int32_t orig = r < rows_t ? p.q_perm[h * p.Nq + prow] : -1;
       const bool valid = orig >= 0 && orig < p.Nq;
       if (r < rows_t && !valid) latch(p.status, EAR_ERR_DEVICE);
-      const bool have_o = ok && c > 0 && mbar_wait_warp(&bars[kBarODone + t], (c - 1) & 1, abort);
+      // the last two chunks' P V (either may still run: nothing later waited on them)
+      bool have_o = ok && c > 0 &&
+                    mbar_wait_warp(&bars[kBarODone + t * kSBufs + ((c - 1) & 1)], ((c - 1) >> 1) & 1,
+                                   abort);
+      if (have_o && c > 1)
+        have_o = mbar_wait_warp(&bars[kBarODone + t * kSBufs + ((c - 2) & 1)], ((c - 2) >> 1) & 1,
+                                abort);
       if (have_o) tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint16_t* orow = p.O + ((int64_t)h * p.Nq + (valid ? orig : 0)) * D;
@@ -678,9 +693,11 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
     mbar_init(&bars[kBarQFull], 1);
     mbar_init(&bars[kBarDrain], 1);
     for (int t = 0; t < kTiles; ++t) {
-      mbar_init(&bars[kBarSFull + t], 1);
-      mbar_init(&bars[kBarPFull + t], kTileRows);
-      mbar_init(&bars[kBarODone + t], 1);
+      for (int b = 0; b < kSBufs; ++b) {
+        mbar_init(&bars[kBarSFull + t * kSBufs + b], 1);
+        mbar_init(&bars[kBarPFull + t * kSBufs + b], kTileRows);
+        mbar_init(&bars[kBarODone + t * kSBufs + b], 1);
+      }
     }
     *abort = 0;
     fence_barrier_init();
