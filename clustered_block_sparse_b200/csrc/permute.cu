@@ -2,14 +2,17 @@
 // out contiguously so the attention map splits into cluster x cluster blocks).
 //
 // A stable counting sort per slice, in 1024-token tiles:
-//  * pm_tile_hist: per (slice, cluster, tile) member counts.
+//  * pm_tile_hist: per (slice, tile, cluster) member counts (cluster fastest,
+//                  so the scan below reads them coalesced).
 //  * pm_scan:      one block per slice turns them into the first output
 //                  position of every (cluster, tile) and writes offsets.
 //  * pm_scatter:   each tile walks its 32 warps in order; a warp groups equal
 //                  labels with __match_any_sync, so a token's position is the
 //                  (cluster, tile) cursor plus the number of earlier tokens of
 //                  its cluster - the order within a cluster is token order.
-//  * pm_gather:    X_perm[r] = X[perm[r]], 16-byte vector copies.
+//  * pm_gather:    X_perm[r] = X[perm[r]], 16-byte vector copies; a warp
+//                  moves several rows at once (lanes split per row) with four
+//                  row groups in flight per thread.
 //  * pm_segmean:   per-cluster fp32 mean of the permuted rows (v̄, §4.3), a
 //                  fixed-order reduction.
 #include "ear_internal.cuh"
@@ -30,7 +33,7 @@ pm_tile_hist(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
     latch(status, EAR_ERR_DEVICE);
     return;
   }
-  atomicAdd(hist + ((h * C + c) * ntiles + blockIdx.x), 1);
+  atomicAdd(hist + ((h * ntiles + blockIdx.x) * C + c), 1);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -40,14 +43,15 @@ pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int nti
   __shared__ int32_t carry;
   const int64_t h = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int32_t* hh = hist + h * (int64_t)C * ntiles;
+  int32_t* hh = hist + h * (int64_t)C * ntiles;  // [tile][cluster]
   int32_t* th = totals + h * (int64_t)C;
-  // per cluster: exclusive prefix over tiles, total in `totals`
+  // per cluster: exclusive prefix over tiles, total in `totals` (consecutive
+  // threads read consecutive clusters of one tile)
   for (int c = tid; c < C; c += 1024) {
     int32_t run = 0;
     for (int t = 0; t < ntiles; ++t) {
-      int32_t v = hh[(int64_t)c * ntiles + t];
-      hh[(int64_t)c * ntiles + t] = run;
+      const int32_t v = hh[(int64_t)t * C + c];
+      hh[(int64_t)t * C + c] = run;
       run += v;
     }
     th[c] = run;
@@ -87,8 +91,8 @@ pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int nti
   __syncthreads();
   // cursor of every (cluster, tile) = cluster offset + earlier tiles' members
   for (int c = tid; c < C; c += 1024) {
-    int32_t o = oh[c];
-    for (int t = 0; t < ntiles; ++t) hh[(int64_t)c * ntiles + t] += o;
+    const int32_t o = oh[c];
+    for (int t = 0; t < ntiles; ++t) hh[(int64_t)t * C + c] += o;
   }
 }
 
@@ -107,7 +111,7 @@ pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
   const unsigned group = __match_any_sync(0xffffffffu, c);
   const int leader = __ffs(group) - 1;
   const int before = __popc(group & ((1u << lane) - 1u));
-  int32_t* cur = cursor + (h * C + (c < 0 ? 0 : c)) * (int64_t)ntiles + tile;
+  int32_t* cur = cursor + (h * ntiles + tile) * (int64_t)C + (c < 0 ? 0 : c);
   for (int w = 0; w < 32; ++w) {
     if (wid == w) {
       int32_t base = 0;
@@ -122,22 +126,37 @@ pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
   }
 }
 
+// row_vecs (16-byte vectors per row) divides 32: 8, 16 or 32
 __global__ void pm_gather(const uint4* __restrict__ X, uint4* __restrict__ Xp,
                           const int32_t* __restrict__ perm, int64_t N, int row_vecs,
                           int64_t rows_total, int* status) {
+  constexpr int kDepth = 4;  // row groups in flight per thread
   const int lane = threadIdx.x & 31;
+  const int groups = 32 / row_vecs;  // rows a warp moves per group
+  const int gi = lane / row_vecs, u = lane % row_vecs;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t g = warp; g < rows_total; g += nwarps) {
-    const int64_t h = g / N;
-    const int32_t src = perm[g];
-    if (src < 0 || src >= N) {
-      if (lane == 0) latch(status, EAR_ERR_DEVICE);
-      continue;
+  const int64_t step = (int64_t)groups * kDepth;
+  for (int64_t base = warp * step; base < rows_total; base += nwarps * step) {
+    uint4 v[kDepth];
+    int64_t dst[kDepth];
+#pragma unroll
+    for (int k = 0; k < kDepth; ++k) {
+      const int64_t g = base + (int64_t)k * groups + gi;
+      dst[k] = -1;
+      if (g < rows_total) {
+        const int32_t src = perm[g];
+        if (src >= 0 && src < N) {
+          v[k] = X[((g / N) * N + src) * row_vecs + u];
+          dst[k] = g * row_vecs + u;
+        } else if (u == 0) {
+          latch(status, EAR_ERR_DEVICE);
+        }
+      }
     }
-    const uint4* s = X + (h * N + src) * row_vecs;
-    uint4* dst = Xp + g * row_vecs;
-    for (int v = lane; v < row_vecs; v += 32) dst[v] = s[v];
+#pragma unroll
+    for (int k = 0; k < kDepth; ++k)
+      if (dst[k] >= 0) Xp[dst[k]] = v[k];
   }
 }
 
