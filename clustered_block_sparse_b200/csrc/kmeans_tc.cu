@@ -147,12 +147,30 @@ __device__ __forceinline__ float group_min(const uint32_t (&v)[32], const float*
   return fminf(fminf(m[0], m[1]), fminf(m[2], m[3]));
 }
 
-// bit k set where d~ of column k is <= thr
+// bit k set where d~ of column k is <= thr (the same packed fma as group_min,
+// so a column's d~ is bit-identical in both)
 __device__ __forceinline__ uint32_t group_hits(const uint32_t (&v)[32], const float* cn, float thr) {
+  const unsigned long long m2 = 0xC0000000C0000000ull;  // (-2.f, -2.f)
+  const float4* c4 = reinterpret_cast<const float4*>(cn);
   uint32_t hit = 0;
 #pragma unroll
-  for (int k = 0; k < 32; ++k)
-    hit |= (fmaf(-2.f, __uint_as_float(v[k]), cn[k]) <= thr ? 1u : 0u) << k;
+  for (int k = 0; k < 32; k += 4) {
+    const float4 cc = c4[k / 4];
+    const unsigned long long c01 =
+        (unsigned long long)__float_as_uint(cc.x) | ((unsigned long long)__float_as_uint(cc.y) << 32);
+    const unsigned long long c23 =
+        (unsigned long long)__float_as_uint(cc.z) | ((unsigned long long)__float_as_uint(cc.w) << 32);
+    const unsigned long long v01 = (unsigned long long)v[k] | ((unsigned long long)v[k + 1] << 32);
+    const unsigned long long v23 =
+        (unsigned long long)v[k + 2] | ((unsigned long long)v[k + 3] << 32);
+    unsigned long long d01, d23;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d01) : "l"(v01), "l"(m2), "l"(c01));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d23) : "l"(v23), "l"(m2), "l"(c23));
+    hit |= (__uint_as_float((uint32_t)d01) <= thr ? 1u : 0u) << k;
+    hit |= (__uint_as_float((uint32_t)(d01 >> 32)) <= thr ? 1u : 0u) << (k + 1);
+    hit |= (__uint_as_float((uint32_t)d23) <= thr ? 1u : 0u) << (k + 2);
+    hit |= (__uint_as_float((uint32_t)(d23 >> 32)) <= thr ? 1u : 0u) << (k + 3);
+  }
   return hit;
 }
 
@@ -332,6 +350,16 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
           if (gmin[u] > thr) continue;
           const int cbase = j * kColChunk + 32 * gg;
           uint32_t hit = group_hits(v, cn + cbase, thr);
+          if ((hit & (hit - 1)) == 0) {
+            // one hit (the usual case): it is the group's minimum column, so
+            // its d~ is gmin[u] and needs no extraction from v
+            if (hit) {
+              c3 = c2; d3 = d2; c2 = c1; d2 = d1; c1 = c0; d1 = d0;
+              c0 = cbase + __ffs(hit) - 1; d0 = gmin[u];
+              ++nc;
+            }
+            hit = 0;
+          }
           while (hit) {
             const int k = __ffs(hit) - 1;
             hit &= hit - 1;

@@ -21,6 +21,16 @@ constexpr int kJ = 64;       // keys per chunk
 constexpr int kClusters = 4; // key clusters per block
 constexpr int kThreads = 256;
 
+__device__ __forceinline__ unsigned long long pk2(float lo, float hi) {
+  return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
@@ -91,23 +101,35 @@ pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
           for (int i = 0; i < 4; ++i) ks[(k0 + i) * kJ + j] = v[i];
         }
         __syncthreads();
-        float acc[8][4];
+        // acc2[ip][j] = (acc[2 ip][j], acc[2 ip + 1][j]): one packed fp32x2 FMA per
+        // centroid pair and key, each lane the same fma sequence over k as a scalar loop
+        unsigned long long acc2[4][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+          for (int j = 0; j < 4; ++j) acc2[i][j] = 0ull;
 #pragma unroll 4
         for (int k = 0; k < D; ++k) {
           const float4 q0 = *reinterpret_cast<const float4*>(qs + k * kA + ty * 8);
           const float4 q1 = *reinterpret_cast<const float4*>(qs + k * kA + ty * 8 + 4);
           const float4 kv = *reinterpret_cast<const float4*>(ks + k * kJ + tx * 4);
-          const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-          const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+          const unsigned long long qp[4] = {pk2(q0.x, q0.y), pk2(q0.z, q0.w), pk2(q1.x, q1.y),
+                                            pk2(q1.z, q1.w)};
+          const unsigned long long kp[4] = {pk2(kv.x, kv.x), pk2(kv.y, kv.y), pk2(kv.z, kv.z),
+                                            pk2(kv.w, kv.w)};
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kk[j], acc[i][j]);
+            for (int j = 0; j < 4; ++j) acc2[i][j] = fma2(qp[i], kp[j], acc2[i][j]);
         }
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[2 * i][j] = __uint_as_float((uint32_t)acc2[i][j]);
+            acc[2 * i + 1][j] = __uint_as_float((uint32_t)(acc2[i][j] >> 32));
+          }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
