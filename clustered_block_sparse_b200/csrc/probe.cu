@@ -10,7 +10,8 @@
 // slice's centroids q̄ transposed in shared memory ([k][a], up to 128 at a
 // time) and walks each cluster's contiguous rows in 64-row chunks, centred
 // and transposed ([k][j]); a thread accumulates an 8 x 4 tile (8 centroids x
-// 4 keys) from one 8-wide and one 4-wide vector load per k.
+// 4 keys) from one 8-wide and one 4-wide vector load per k, as packed fp32x2
+// FMAs on centroid pairs (each element the same fma sequence over k).
 #include "ear_internal.cuh"
 
 namespace ear {

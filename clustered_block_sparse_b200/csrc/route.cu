@@ -12,7 +12,7 @@
 // digit at which the running cost crosses the remaining budget.  Ratios are
 // correctly rounded fp64 divisions, so the order matches a host fp64 sort.
 //
-// Main path (C_q C_k <= 8 x kKeysPerCta): one cluster of 8 CTAs per slice.
+// Main path (C_q <= 1024 and C_q C_k <= 8 x kKeysPerCta): one cluster of 8 CTAs per slice.
 // Each CTA keeps the keys of its eighth of the blocks in shared memory; in
 // each pass every CTA adds its costs into the histogram of CTA 0 through
 // distributed shared memory (a warp whose lanes share one digit adds them in
