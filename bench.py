@@ -199,7 +199,7 @@ def recorded_traffic(heads: int):
     import hashlib
 
     here = os.path.dirname(os.path.abspath(__file__))
-    prof = os.path.join(here, "profiles", "attention_tc_wan.md")
+    prof = os.path.join(here, "profiles", "attention_tc_wan.txt")
     src = os.path.join(here, "clustered_block_sparse_b200", "csrc", "attention_tc.cu")
     try:
         text = open(prof).read()
@@ -354,7 +354,7 @@ def run_ear(args, w):
                      "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)",
                      "traffic": recorded_traffic(w.heads),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                       "at_tc at 4 heads (profiles/attention_tc_wan.md), "
+                                       "at_tc at 4 heads (profiles/attention_tc_wan.txt), "
                                        "scaled by heads; null if the kernel changed since",
                      "algorithmic_bytes": attention_bytes(w),
                      "algorithmic_flops": fl["attention"]},

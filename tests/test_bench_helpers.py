@@ -27,7 +27,7 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path):
     src = csrc / "attention_tc.cu"
     src.write_text("// kernel v1\n")
     sha = hashlib.sha256(src.read_bytes()).hexdigest()
-    (tmp_path / "profiles" / "attention_tc_wan.md").write_text(
+    (tmp_path / "profiles" / "attention_tc_wan.txt").write_text(
         f"summary\n\ntraffic_bytes_per_head: 1000\nkernel_source_sha256: {sha}\n")
     bench = _load_bench(str(tmp_path / "bench.py"))
     assert bench.recorded_traffic(40) == 40000
