@@ -17,7 +17,7 @@ EAR_OP_KMEANS, EAR_OP_PERMUTE, EAR_OP_PROBE, EAR_OP_ROUTE, EAR_OP_ATTENTION = ra
 EAR_COMPENSATE = 1
 
 EXPORTED = ("ear_status_string", "ear_workspace_bytes", "ear_kmeans", "ear_permute",
-            "ear_permute_static", "ear_probe", "ear_route", "ear_attention",
+            "ear_permute_apply", "ear_permute_static", "ear_probe", "ear_route", "ear_attention",
             "ear_get_device_status", "ear_launch_count")
 PERMUTE_STATIC_MAX_BYTES = 8 << 20
 
@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
                              _vp, ctypes.c_size_t, _vp]
     L.ear_permute.argtypes = [_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_int, _i32, _vp,
                               _vp, ctypes.c_size_t, _vp]
+    L.ear_permute_apply.argtypes = [_vp, _vp, _i64, _i64, _i32, _vp, _vp, ctypes.c_int, _i32, _vp,
+                                    _vp]
     L.ear_permute_static.argtypes = [_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_int,
                                      _i32, _vp, _vp]
     L.ear_probe.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _vp, _i64, _i64, _i32, _i32, _i32,
@@ -62,7 +64,8 @@ def lib() -> ctypes.CDLL:
     L.ear_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), _vp]
     L.ear_launch_count.argtypes = []
     L.ear_launch_count.restype = ctypes.c_uint64
-    for name in ("ear_workspace_bytes", "ear_kmeans", "ear_permute", "ear_permute_static",
+    for name in ("ear_workspace_bytes", "ear_kmeans", "ear_permute", "ear_permute_apply",
+                 "ear_permute_static",
                  "ear_probe", "ear_route",
                  "ear_attention", "ear_get_device_status"):
         getattr(L, name).restype = ctypes.c_int

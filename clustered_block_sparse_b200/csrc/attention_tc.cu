@@ -8,8 +8,14 @@
 //   * exact boxes: the rows of every key cluster b listed for a, 32 at a
 //     time (the last box of a cluster is partial), so small clusters share
 //     a chunk instead of each paying for a whole MMA round;
-//   * compensation boxes (EAR_COMPENSATE): the C_k key / value centroids, 32
-//     at a time, with per-column bias log2|b| (weight |b|) and -inf for
+//   * compensation chunks (EAR_COMPENSATE): the C_k key / value centroids, 32
+//     at a time, each held as two bf16 boxes (hi = bf16(x), lo = bf16(x - hi),
+//     16 significant bits together).  To the MMA issuer such a chunk is a
+//     64-key chunk whose keys 0-31 are the hi rows and 32-63 the lo rows: the
+//     softmax adds the two halves of S in fp32 (s q·k̄ = S_hi + S_lo) and writes
+//     the same P for both halves, so P V adds P v̄_hi + P v̄_lo.  The
+//     compensated logits and values thus keep the fp32 centroids to about
+//     2^-17 relative.  The per-column bias is log2|b| (weight |b|), -inf for
 //     clusters that are exact for a or empty.  Exact and centroid boxes never
 //     share a chunk.
 // Warp roles (12 warps):
@@ -55,13 +61,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // move the running max only when it grows by > 2^8
 constexpr int kTableMax = 2048;   // block list / key offsets staged in shared memory up to this
 // Register split (setmaxnreg): warps 0-3 (producer, MMA issuer, 2 idle) drop
-// to kRegsLow, the two softmax warpgroups rise to kRegsHigh.  The sum stays
+// to regs_low<D>(), the two softmax warpgroups rise to kRegsHigh.  The sum stays
 // within the 168 registers x 384 threads the kernel is launched with; the
 // launcher checks the compiled count before every launch.
-constexpr int kRegsLow = 64;
+template <int D>
+constexpr int regs_low() { return D == 128 ? 72 : 64; }
 constexpr int kRegsHigh = 216;
 constexpr int kRegsLaunch = 168;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
+static_assert(128 * regs_low<128>() + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
+static_assert(128 * regs_low<64>() + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 // barrier slots
 constexpr int kBarKvFull = 0;                     // + stage
@@ -96,7 +104,8 @@ struct Layout {
   static constexpr int kInfo = kBias + kStages * kChunk * 4;    // [stage] ChunkInfo
   static constexpr int kList = kInfo + kStages * 32;              // unit's exact key clusters
   static constexpr int kKoff = kList + kTableMax * 4;             // slice's key offsets
-  static constexpr int kBar = kKoff + kTableMax * 4;
+  static constexpr int kExact = kKoff + kTableMax * 4;            // unit's row of the mask
+  static constexpr int kBar = kExact + kTableMax;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -167,7 +176,7 @@ struct Boxes {
       return true;
     }
     if (compensate && comp_next < Ck) {
-      row = comp_next;
+      row = comp_next;  // centroid index; its hi / lo boxes sit at rows 2 row, 2 row + 32
       valid = min(kBox, Ck - comp_next);
       comp_next += kBox;
       comp = true;
@@ -222,16 +231,17 @@ __device__ __forceinline__ float box_max_bias(const uint32_t (&v)[32], const flo
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// p = 2^(score * scale + shift_j) for 32 columns (shift pairs from `sh`),
-// packed to bf16 pairs; returns the two partial row sums as a pair.
-__device__ __forceinline__ unsigned long long box_exp(const uint32_t (&v)[32],
-                                                      const unsigned long long (&sh)[16],
-                                                      unsigned long long scale2, int valid,
-                                                      uint32_t (&pk)[16]) {
+// p = 2^(score * scale + bias_j - m) for 32 columns (bias from shared memory,
+// neg = -m), packed to bf16 pairs; returns the two partial row sums as a pair.
+__device__ __forceinline__ unsigned long long box_exp(const uint32_t (&v)[32], const float* bias,
+                                                      float neg, unsigned long long scale2,
+                                                      int valid, uint32_t (&pk)[16]) {
   unsigned long long sum = 0;
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    const unsigned long long z = fma2(pack2(v[j], v[j + 1]), scale2, sh[j / 2]);
+    const float2 b2 = *reinterpret_cast<const float2*>(bias + j);
+    const unsigned long long sh = pack2(__float_as_uint(b2.x + neg), __float_as_uint(b2.y + neg));
+    const unsigned long long z = fma2(pack2(v[j], v[j + 1]), scale2, sh);
     float p0 = ex2(lo_f(z)), p1 = ex2(hi_f(z));
     if (valid < 32) {
       p0 = j < valid ? p0 : 0.f;
@@ -295,14 +305,18 @@ __device__ __forceinline__ void producer_role(
     const int32_t* glist = p.blk_list + h * (int64_t)p.Cq * p.Ck + e0;
     const int32_t* list = glist;
     const int32_t* koff_t = koff;
+    const uint8_t* exact_t = exact_row;
     if (nlist <= kTableMax && p.Ck + 1 <= kTableMax && nlist >= 0) {
       int32_t* sl = reinterpret_cast<int32_t*>(smem + L::kList);
       int32_t* sk = reinterpret_cast<int32_t*>(smem + L::kKoff);
+      uint8_t* se = smem + L::kExact;
       for (int i = lane; i < nlist; i += 32) sl[i] = glist[i];
       for (int i = lane; i <= p.Ck; i += 32) sk[i] = koff[i];
+      for (int i = lane; i < p.Ck; i += 32) se[i] = exact_row[i];
       __syncwarp();
       list = sl;
       koff_t = sk;
+      exact_t = se;
     }
     Boxes it;
     it.init(p, list, max(nlist, 0), koff_t);
@@ -324,6 +338,7 @@ __device__ __forceinline__ void producer_role(
 #pragma unroll
       for (int k = 0; k < kBoxes; ++k) {
         if (!(have && (bcomp ? 1 : 0) == comp)) break;
+        if (k > 0 && comp) break;  // a centroid chunk is one group of 32 (hi + lo boxes)
         if (k == 0) { r0 = brow; v0 = bval; }
         if (k == 1) { r1 = brow; v1 = bval; }
         nbox = k + 1;
@@ -345,7 +360,7 @@ __device__ __forceinline__ void producer_role(
           if (bx < nbox && (j % kBox) < vb) {
             const int b = comp_first + j;
             const int32_t cnt = koff_t[b + 1] - koff_t[b];
-            if (!exact_row[b] && cnt > 0) bv = __log2f((float)cnt);
+            if (!exact_t[b] && cnt > 0) bv = __log2f((float)cnt);
           }
           bias[s * kChunk + j] = bv;
         }
@@ -360,20 +375,21 @@ __device__ __forceinline__ void producer_role(
         if (nbox == 0)
           mbar_arrive(&bars[kBarKvFull + s]);  // end of the sequence
         else
-          mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * nbox * kBox * D * 2);
+          mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * (comp ? 2 : nbox) * kBox * D * 2);
       }
       {
         const CUtensorMap* mk = comp ? &tmKc : &tmK;
         const CUtensorMap* mv = comp ? &tmVc : &tmV;
         const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
+        const int nphys = comp ? 2 : nbox;  // a centroid chunk loads its hi and lo boxes
         uint8_t* kdst = smem + L::kK + s * L::kStageBytes;
         uint8_t* vdst = smem + L::kV + s * L::kStageBytes;
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
-          const int32_t rw = bx == 0 ? r0 : r1;
+          const int32_t rw = comp ? 2 * r0 + bx * kBox : (bx == 0 ? r0 : r1);
 #pragma unroll
           for (int hf = 0; hf < D / 64; ++hf) {
-            if (bx < nbox && leader) {
+            if (bx < nphys && leader) {
               tma_load_2d(kdst + hf * L::kSHalf + bx * kBox * 128, mk, &bars[kBarKvFull + s],
                           64 * hf, base + rw);
               tma_load_2d(vdst + hf * L::kSHalf + bx * kBox * 128, mv, &bars[kBarKvFull + s],
@@ -408,6 +424,7 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
       const bool leader = elect_one();
       const uint32_t idesc_pv = idesc_bf16(128, D, true);
       // S of tile t, buffer b: TMEM columns [128 t + 64 b, +64); O_t: [256 + 128 t, +128)
+      // n = keys of the chunk (32 or 64; a centroid chunk is 64: hi rows, then lo rows)
       auto issue_qk = [&](int t, int buf, int s, int n) {
         const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
         const uint64_t qd = desc_sw128(smem_u32(smem + L::kQ + t * L::kTileBytes), 16, 1024);
@@ -437,7 +454,9 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
       // n0, n1: keys of chunks c and c+1 (0 = past the end)
       bool ok = mbar_wait_warp(&bars[kBarQFull], 0, abort) &&
                 mbar_wait_warp(&bars[kBarKvFull], 0, abort);
-      int n0 = ok ? info[0].nbox * kBox : 0, n1 = 0;
+      // n0, n1: keys of chunks c and c+1 (0 = past the end)
+      auto keys_of = [&](int st) { return (info[st].comp ? 2 : info[st].nbox) * kBox; };
+      int n0 = ok ? keys_of(0) : 0, n1 = 0;
       if (ok && n0 > 0) {
         tc_fence_after();
         for (int t = 0; t < ntiles; ++t) {
@@ -445,7 +464,7 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
           commit(&bars[kBarSFull + t * kSBufs]);
         }
         ok = mbar_wait_warp(&bars[kBarKvFull + 1], 0, abort);
-        n1 = ok ? info[1].nbox * kBox : 0;
+        n1 = ok ? keys_of(1) : 0;
         if (ok && n1 > 0) {
           tc_fence_after();
           for (int t = 0; t < ntiles; ++t) {
@@ -468,7 +487,7 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
           if (t == 0 && n1 > 0) {
             ok = mbar_wait_warp(&bars[kBarKvFull + s2], ((c + 2) / kStages) & 1, abort);
             if (!ok) break;
-            n2 = info[s2].nbox * kBox;
+            n2 = keys_of(s2);
             tc_fence_after();
           }
           if (n2 > 0) {  // chunk c+2 into the buffer P V of chunk c has just read
@@ -553,18 +572,17 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
             tmem_st16(tS + 16, pk);
           }
         } else {
-          // centroid chunk, pass 1: chunk max (scaled, with the bias)
-          float mx = -INFINITY;
-          for (int bx = 0; bx < nbox; bx += 2) {
-            uint32_t va[32], vb[32];
-            const bool has_b = bx + 1 < nbox;
-            tmem_ld32(tS + 32 * bx, va);
-            if (has_b) tmem_ld32(tS + 32 * (bx + 1), vb);
-            tmem_ld_wait();
-            const int v0 = ci->valid[bx], v1 = has_b ? ci->valid[bx + 1] : 0;
-            mx = fmaxf(mx, box_max_bias(va, bs + 32 * bx, scale, v0));
-            if (has_b) mx = fmaxf(mx, box_max_bias(vb, bs + 32 * (bx + 1), scale, v1));
-          }
+          // centroid chunk: S columns 0-31 = Q k̄_hi^T, 32-63 = Q k̄_lo^T for 32
+          // centroids; s q·k̄ = S_hi + S_lo in fp32, weight |b| through the bias
+          const int v0 = ci->valid[0];
+          uint32_t x0[32], x1[32];
+          tmem_ld32(tS, x0);
+          tmem_ld32(tS + 32, x1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            x0[j] = __float_as_uint(__uint_as_float(x0[j]) + __uint_as_float(x1[j]));
+          const float mx = box_max_bias(x0, bs, scale, v0);
           if (mx > m + kRescale || (m == -INFINITY && mx > -INFINITY)) {
             if (m != -INFINITY) {
               resc = true;
@@ -573,22 +591,11 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
             m_use = mx;
           }
           if (resc) lsum = pack2(__float_as_uint(lo_f(lsum) * corr), __float_as_uint(hi_f(lsum) * corr));
-          // centroid chunk, pass 2: P = 2^(scaled score + bias - m_use) into the first half of S
           const float neg = m_use == -INFINITY ? 0.f : -m_use;  // all scores -inf: p = 0 below
-          for (int bx = 0; bx < nbox; ++bx) {
-            uint32_t v[32];
-            tmem_ld32(tS + 32 * bx, v);
-            tmem_ld_wait();
-            unsigned long long sh[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              sh[j] = pack2(__float_as_uint(bs[32 * bx + 2 * j] + neg),
-                            __float_as_uint(bs[32 * bx + 2 * j + 1] + neg));
-            const int valid = m_use == -INFINITY ? 0 : ci->valid[bx];
-            uint32_t pk[16];
-            lsum = add2(lsum, box_exp(v, sh, scale2, valid, pk));
-            tmem_st16(tS + 16 * bx, pk);
-          }
+          uint32_t pk[16];
+          lsum = add2(lsum, box_exp(x0, bs, neg, scale2, m_use == -INFINITY ? 0 : v0, pk));
+          tmem_st16(tS, pk);       // P for the hi rows
+          tmem_st16(tS + 16, pk);  // the same P for the lo rows
         }
         tmem_st_wait();
         if (__any_sync(0xffffffffu, resc)) {
@@ -714,7 +721,7 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
   // Each role ends with its own teardown (a CTA-wide bar.sync, then warp 0
   // frees TMEM), so no code runs under both register budgets.
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsLow));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(regs_low<D>()));
     if (warp == 0) {
       producer_role<D>(tmQ, tmK, tmV, tmKc, tmVc, p, smem, h, a, row0, ntiles, lane, abort);
     } else if (warp == 1) {
@@ -735,18 +742,29 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
   asm volatile("bar.sync 0;" ::: "memory");
 }
 
+// Key / value centroids as bf16 pairs: per slice, groups of 32 centroids, each
+// group 32 rows of hi = bf16(x) followed by 32 rows of lo = bf16(x - hi)
+// (x - hi is exact in fp32); rows past C_k are zero.  rows = 64 per group.
 __global__ void at_centroids_bf16(const float* __restrict__ kc, const float* __restrict__ vc,
                                   uint16_t* __restrict__ kc16, uint16_t* __restrict__ vc16,
-                                  int Ck, int Ck_pad, int D, int64_t total) {
+                                  int Ck, int rows, int D, int64_t total) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= total) return;
-  const int64_t hc = e / D;
+  const int64_t hr = e / D;
   const int k = (int)(e % D);
-  const int64_t h = hc / Ck_pad;
-  const int c = (int)(hc % Ck_pad);
-  const bool ok = c < Ck;
-  kc16[e] = ok ? f32_to_bf16(kc[(h * Ck + c) * D + k]) : 0;
-  vc16[e] = ok ? f32_to_bf16(vc[(h * Ck + c) * D + k]) : 0;
+  const int64_t h = hr / rows;
+  const int r = (int)(hr % rows);
+  const int c = (r / 64) * 32 + (r % 32);
+  const bool lo = (r % 64) >= 32;
+  uint16_t ko = 0, vo = 0;
+  if (c < Ck) {
+    const float kx = kc[(h * Ck + c) * D + k], vx = vc[(h * Ck + c) * D + k];
+    const uint16_t kh = f32_to_bf16(kx), vh = f32_to_bf16(vx);
+    ko = lo ? f32_to_bf16(kx - bf16_to_f32(kh)) : kh;
+    vo = lo ? f32_to_bf16(vx - bf16_to_f32(vh)) : vh;
+  }
+  kc16[e] = ko;
+  vc16[e] = vo;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -821,7 +839,7 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
   // refuse to launch a build whose allocation does not.
   cudaFuncAttributes fa;
   EAR_CUDA(cudaFuncGetAttributes(&fa, at_tc<D>));
-  if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh) return EAR_ERR_UNSUPPORTED;
+  if (fa.numRegs * kThreads < 128 * regs_low<D>() + 256 * kRegsHigh) return EAR_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)max_items, (unsigned)a.bh);
   at_tc<D><<<grid, kThreads, L::kBytes, s>>>(mq, mk, mv, mkc, mvc, p);
   return after_launch();
@@ -829,7 +847,8 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
 
 }  // namespace
 
-int64_t attention_tc_ck_pad(int32_t c_k) { return ceil_div(c_k, kChunk) * kChunk; }
+// Rows of the bf16 centroid buffer per slice: 64 (32 hi + 32 lo) per group of 32.
+int64_t attention_tc_ck_pad(int32_t c_k) { return ceil_div(c_k, kBox) * 2 * kBox; }
 
 int64_t attention_tc_items_per_slice(int64_t n_q, int32_t c_q) {
   return ceil_div(n_q, kUnitRows) + c_q;

@@ -3,7 +3,6 @@
 // is enqueued, so a rejected call has no side effect.
 #include <atomic>
 #include <cmath>
-#include <mutex>
 
 #include "ear_internal.cuh"
 
@@ -12,10 +11,6 @@ namespace {
 __device__ int g_status_word;  // first device-side error latched since the last read
 
 std::atomic<uint64_t> g_launches{0};
-
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {nullptr};
-std::mutex g_status_mu;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
@@ -36,16 +31,15 @@ ear_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 namespace ear {
 
+// Looked up on every call rather than cached: after a device reset the module
+// is loaded again at a new address in the new context, and a cached pointer
+// would be stale.  The lookup is a host-side table read once the module is
+// loaded (the first call on a device loads it; make that call before any
+// stream capture begins).
 int* device_status_word() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_status_mu);
-  if (g_status_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_status_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 ear_status after_launch() {
@@ -119,6 +113,19 @@ ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int32_t c,
   if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
   return ear::permute_run(labels, bh, n, c, perm, offsets, X, X_perm, dtype, d, seg_mean, ws,
                           static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_t bh, int64_t n,
+                             int32_t c, const void* X, void* X_perm, ear_dtype dtype, int32_t d,
+                             float* seg_mean, void* stream) {
+  if (bh < 1 || n < 1 || n > kMaxN || c < 1) return EAR_ERR_ARG;
+  if (!ok_ptr(perm) || !ok_ptr(offsets) || !ok_ptr(X) || !ok_ptr(X_perm) || !ok_dtype(dtype))
+    return EAR_ERR_ARG;
+  if (seg_mean != nullptr && !aligned16(seg_mean)) return EAR_ERR_ARG;
+  if (c > kMaxC || bh > kMaxBH || !ok_d(d)) return EAR_ERR_UNSUPPORTED;
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::permute_apply_run(perm, offsets, bh, n, c, X, X_perm, dtype, d, seg_mean,
+                                static_cast<cudaStream_t>(stream));
 }
 
 ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,

@@ -65,8 +65,18 @@ size_t permute_workspace(int64_t bh, int64_t n, int32_t c);
 ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, int32_t* perm,
                        int32_t* offsets, const void* X, void* X_perm, ear_dtype dt, int32_t d,
                        float* seg_mean, void* ws, cudaStream_t s);
+// X_perm[r] = X[perm[r]] and the optional per-cluster means, from a given
+// permutation and its offsets (no workspace).
+ear_status permute_apply_run(const int32_t* perm, const int32_t* offsets, int64_t bh, int64_t n,
+                             int32_t c, const void* X, void* X_perm, ear_dtype dt, int32_t d,
+                             float* seg_mean, cudaStream_t s);
 
 size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
+// Tensor-core probe (bf16 keys).
+size_t probe_tc_workspace(int64_t bh, int32_t d, int32_t c_q, int32_t c_k);
+ear_status probe_tc_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
+                        const int32_t* koff, int64_t bh, int64_t n_k, int32_t d, int32_t c_q,
+                        int32_t c_k, float scale, float* E, void* ws, cudaStream_t s);
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                      ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
                      int32_t c_q, int32_t c_k, float scale, float* E, void* ws, cudaStream_t s);

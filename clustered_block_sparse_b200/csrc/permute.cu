@@ -164,7 +164,7 @@ __global__ void pm_gather(const uint4* __restrict__ X, uint4* __restrict__ Xp,
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 pm_segmean(const T* __restrict__ Xp, const int32_t* __restrict__ offsets, int64_t N, int C,
-           float* __restrict__ mean) {
+           float* __restrict__ mean, int* status) {
   constexpr int kQuads = D / 4;
   constexpr int kGroups = 256 / kQuads;
   __shared__ float4 part[kGroups][kQuads];
@@ -172,7 +172,11 @@ pm_segmean(const T* __restrict__ Xp, const int32_t* __restrict__ offsets, int64_
   const int c = blockIdx.x;
   const int q = threadIdx.x % kQuads, g = threadIdx.x / kQuads;
   const int32_t* oh = offsets + h * (int64_t)(C + 1);
-  const int32_t r0 = oh[c], r1 = oh[c + 1];
+  int32_t r0 = oh[c], r1 = oh[c + 1];
+  if (r0 < 0 || r1 < r0 || r1 > N) {  // offsets passed in by the caller: checked
+    if (threadIdx.x == 0) latch(status, EAR_ERR_DEVICE);
+    r0 = r1 = 0;
+  }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const T* xh = Xp + h * N * D;
   for (int64_t r = r0 + g; r < r1; r += kGroups) {
@@ -219,7 +223,7 @@ template <typename T, int D>
 ear_status segmean_t(const void* Xp, const int32_t* offsets, int64_t bh, int64_t n, int32_t c,
                      float* mean, cudaStream_t s) {
   pm_segmean<T, D><<<dim3((unsigned)c, (unsigned)bh), 256, 0, s>>>((const T*)Xp, offsets, n, c,
-                                                                   mean);
+                                                                   mean, device_status_word());
   return after_launch();
 }
 
@@ -248,6 +252,13 @@ ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, 
   pm_scatter<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, perm);
   EAR_TRY(after_launch());
   if (X == nullptr) return EAR_OK;
+  return permute_apply_run(perm, offsets, bh, n, c, X, X_perm, dt, d, seg_mean, s);
+}
+
+ear_status permute_apply_run(const int32_t* perm, const int32_t* offsets, int64_t bh, int64_t n,
+                             int32_t c, const void* X, void* X_perm, ear_dtype dt, int32_t d,
+                             float* seg_mean, cudaStream_t s) {
+  int* status = device_status_word();
   const int elem = dt == EAR_F32 ? 4 : 2;
   const int row_vecs = d * elem / 16;
   const int64_t rows_total = bh * n;

@@ -6,11 +6,11 @@
 // lives in one fixed-size array compiled into this library.
 //
 // The array is a file-scope __device__ variable, so host code cannot use its
-// name as a device pointer.  Its device address is looked up once per device
-// with cudaGetSymbolAddress (on the first call made on that device, with that
-// device current) and handed to the kernels as their workspace.
-#include <mutex>
-
+// name as a device pointer.  Its device address on the current device is
+// looked up with cudaGetSymbolAddress on every call (the first call on a
+// device loads the module there, so make it before any stream capture) and
+// handed to the kernels as their workspace.  It is not cached: after a device
+// reset the module is loaded again at a new address.
 #include "ear_internal.cuh"
 
 namespace {
@@ -20,22 +20,12 @@ constexpr size_t kScratchBytes = EAR_PERMUTE_STATIC_MAX_BYTES;
 // Kept by every device that loads the library until the process exits.
 static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-std::mutex g_scratch_mu;
-
-// Device address of g_permute_scratch on the current device, looked up once.
+// Device address of g_permute_scratch on the current device.
 ear_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EAR_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
-      return EAR_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
+    return EAR_ERR_CUDA;
+  *out = p;
   return EAR_OK;
 }
 

@@ -1,5 +1,6 @@
-// Compensation-error probe (SVG-EAR §4.2 "Error estimation"; §1: query
-// centroids stand in for the queries of their cluster).
+// Compensation-error probe for fp32 keys (SVG-EAR §4.2 "Error estimation";
+// §1: query centroids stand in for the queries of their cluster).  bf16 keys
+// take the tensor-core kernel in probe_tc.cu.
 //
 //   E[a][b] = sum_{j in b} (s q̄_a·k_j - s q̄_a·k̄_b)^2 = sum_{j in b} (s q̄_a·(k_j - k̄_b))^2
 //
@@ -168,16 +169,18 @@ ear_status run_t(const float* qc, const int32_t* qn, const float* kc, const void
 
 }  // namespace
 
-size_t probe_workspace(int64_t, int64_t, int32_t, int32_t, int32_t) { return 0; }
+// bf16 keys run on the tensor cores (probe_tc.cu); fp32 keys here.
+size_t probe_workspace(int64_t bh, int64_t, int32_t d, int32_t c_q, int32_t c_k) {
+  return probe_tc_workspace(bh, d, c_q, c_k);
+}
 
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                      ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, float* E, void*, cudaStream_t s) {
-  if (dt == EAR_F32)
-    return d == 64 ? run_t<float, 64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s)
-                   : run_t<float, 128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s);
-  return d == 64 ? run_t<uint16_t, 64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s)
-                 : run_t<uint16_t, 128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s);
+                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws, cudaStream_t s) {
+  if (dt == EAR_BF16)
+    return probe_tc_run(qc, qn, kc, K, koff, bh, n_k, d, c_q, c_k, scale, E, ws, s);
+  return d == 64 ? run_t<float, 64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s)
+                 : run_t<float, 128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s);
 }
 
 }  // namespace ear

@@ -91,6 +91,24 @@ def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor]
     return perm, offsets, x_perm, mean
 
 
+def ear_permute_apply(perm: torch.Tensor, offsets: torch.Tensor, x: torch.Tensor,
+                      seg_mean: bool = False):
+    """X_perm[r] = X[perm[r]] with a permutation made by ear_permute, plus the
+    optional per-cluster means (SVG-EAR §4.3: V in K's cluster order, v̄).
+
+    Returns (x_perm, mean [BH,C,d] f32 or None)."""
+    for t, nm in ((perm, "perm"), (offsets, "offsets"), (x, "x")):
+        _need(t, nm)
+    bh, n, d = x.shape
+    c = offsets.shape[1] - 1
+    x_perm = torch.empty_like(x)
+    mean = torch.empty((bh, c, d), dtype=torch.float32, device=x.device) if seg_mean else None
+    N.check("ear_permute_apply", N.lib().ear_permute_apply(
+        _p(perm), _p(offsets), bh, n, c, _p(x), _p(x_perm), _dtype(x), d, _p(mean),
+        _stream(x.device)))
+    return x_perm, mean
+
+
 def ear_permute_static(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor] = None,
                        seg_mean: bool = False):
     """ear_permute without a workspace, for callers that cannot allocate device
@@ -221,7 +239,7 @@ def ear_layer(q, k, v, q_init, k_init, iters: int, density: float, ratio_mode: i
     kc, kl, kn = ear_kmeans(k, k_init, iters)
     qp, qo, qx, _ = ear_permute(ql, q_init.shape[1], q)
     kp, ko, kx, _ = ear_permute(kl, k_init.shape[1], k)
-    _, _, vx, vm = ear_permute(kl, k_init.shape[1], v, seg_mean=True)
+    vx, vm = ear_permute_apply(kp, ko, v, seg_mean=True)
     e = ear_probe(qc, qn, kc, kx, ko, scale)
     exact, bo, bl, pairs = ear_route(e, qn, kn, n_q, n_k, density, ratio_mode)
     o, lse = ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, scale, compensate,

@@ -8,8 +8,8 @@
  * One attention layer runs five calls, in this order, for all (batch, head)
  * slices at once ("BH" slices):
  *   ear_kmeans(Q), ear_kmeans(K)       cluster queries and keys
- *   ear_permute(Q), (K), (V with K's   make each cluster contiguous
- *     labels, also producing v̄)
+ *   ear_permute(Q), (K)                make each cluster contiguous
+ *   ear_permute_apply(V, K's perm)     V in K's order, also producing v̄
  *   ear_probe                          per-block compensation-error estimate
  *   ear_route                          greedy error-to-cost block selection
  *   ear_attention                      block-sparse exact attention plus
@@ -134,6 +134,24 @@ EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int
                        void* stream);
 
 /*
+ * Applies a permutation made by ear_permute to another token matrix (SVG-EAR
+ * §4.3: V follows the key clustering, so V is laid out with K's permutation
+ * and v̄_b is the mean of V over key cluster b).  No labels are recounted.
+ *   perm     [BH][N] int32          from ear_permute (a bijection of [0, N))
+ *   offsets  [BH][C+1] int32        from the same call
+ *   X        [BH][N][d] dtype       rows in original order
+ *   X_perm   [BH][N][d] dtype  out  X_perm[r] = X[perm[r]]
+ *   seg_mean [BH][C][d] float  out  optional mean of X's rows of each cluster
+ *                                   (rows offsets[c] .. offsets[c+1]-1 of
+ *                                   X_perm); zero rows for empty clusters
+ * Takes no workspace.  A perm entry outside [0, N) latches EAR_ERR_DEVICE and
+ * that row is not written.
+ */
+EAR_API ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_t bh,
+                                     int64_t n, int32_t c, const void* X, void* X_perm,
+                                     ear_dtype dtype, int32_t d, float* seg_mean, void* stream);
+
+/*
  * ear_permute_static - ear_permute for callers that cannot allocate device
  * memory (the paper has no counterpart: this is a deployment variant).
  *
@@ -148,9 +166,10 @@ EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int
  *     reports; a problem needing more than EAR_PERMUTE_STATIC_MAX_BYTES is
  *     rejected with EAR_ERR_WORKSPACE before anything runs.  (8 MiB holds,
  *     e.g., 40 slices of 75,600 tokens in 500 clusters.)
- *   - The first call on a device looks up the array's device address on
- *     that device (the device must be current); make that first call before
- *     any stream capture begins.
+ *   - Every call looks up the array's device address on the current device
+ *     (so a device reset between calls is safe); the first call on a device
+ *     also loads the library's GPU code there, so make it before any stream
+ *     capture begins.
  *   - No call allocates or frees memory (no cudaMalloc / cudaFree).
  *   - Every call reuses the same array and leaves its contents behind; each
  *     call clears what it needs zeroed.  Calls whose work overlaps on the

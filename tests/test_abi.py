@@ -89,6 +89,14 @@ def test_permute_validation(lib):
     assert f(FAKE, 1, 100, 4, FAKE, FAKE, None, None, 0, 0, None, FAKE, 4, None) == N.EAR_ERR_WORKSPACE
 
 
+def test_permute_apply_validation(lib):
+    f = lib.ear_permute_apply
+    assert f(None, FAKE, 1, 100, 4, FAKE, FAKE, 1, 128, None, None) == N.EAR_ERR_ARG
+    assert f(FAKE, FAKE, 1, 100, 4, None, FAKE, 1, 128, None, None) == N.EAR_ERR_ARG
+    assert f(FAKE, FAKE, 1, 100, 4, FAKE, FAKE, 1, 128, MISALIGNED, None) == N.EAR_ERR_ARG
+    assert f(FAKE, FAKE, 1, 100, 4, FAKE, FAKE, 1, 96, None, None) == N.EAR_ERR_UNSUPPORTED
+
+
 def test_probe_validation(lib):
     f = lib.ear_probe
     assert f(FAKE, FAKE, FAKE, FAKE, 1, FAKE, 1, 100, 128, 4, 4, ctypes.c_float(float("nan")),

@@ -157,6 +157,25 @@ def test_permute_matches_oracle(n, c, dtype, d):
         np.testing.assert_allclose(mean[h], m_ref, rtol=0, atol=1e-6 * max(np.abs(m_ref).max(), 1))
 
 
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_permute_apply_reuses_a_permutation(dtype, d):
+    """V laid out with K's permutation (no recount) equals the oracle's gather
+    and segment means."""
+    rng = np.random.default_rng(11)
+    bh, n, c = 2, 3001, 41
+    labels = rng.integers(0, c, (bh, n)).astype(np.int32)
+    labels[labels == 5] = 6  # an empty cluster
+    v = gen.round_to_dtype(rng.standard_normal((bh, n, d)), dtype)
+    perm, off, _, _ = ear.ear_permute(pu.dev(labels), c)
+    vp, mean = ear.ear_permute_apply(perm, off, pu.dev(v, pu.torch_dtype(dtype)), seg_mean=True)
+    vp, mean = pu.host(vp), pu.host(mean)
+    for h in range(bh):
+        p_ref, _ = eo.permute(labels[h], c)
+        np.testing.assert_array_equal(vp[h], v[h][p_ref])
+        m_ref = eo.segment_mean(v[h], labels[h], c)
+        np.testing.assert_allclose(mean[h], m_ref, rtol=0, atol=1e-6 * max(np.abs(m_ref).max(), 1))
+
+
 def test_permute_bad_label_latches_device_status():
     labels = np.zeros((1, 100), np.int32)
     labels[0, 17] = 9  # out of range for C = 4
@@ -432,3 +451,153 @@ def test_wan_layer_full_size_sampled():
         vm = eo.segment_mean(L.v[h], klab, w.c_k)
         o_ref, _ = eo.attention(L.q[h][qi], L.k[h], L.v[h], qlab[qi], klab, kc, vm, kn, ex_ref, s)
         pu.assert_attention_close(o[h][qi], o_ref, "bf16")
+
+
+# --------------------------------------------------------------------------- probe -> route
+def _probe_route_case(q, k, qi, ki, iters, d, densities, dtype):
+    """Oracle k-means and permutation; then ear_probe and ear_route on the GPU
+    from the oracle's centroids (rounded to fp32, the ABI's type), counts and
+    permuted keys, against eo.route(eo.probe(...)) on the same values.  A
+    routed block may differ only at a ratio tie within 1e-6 of the oracle's
+    cut; the lists, offsets and pair count must describe the GPU's own mask."""
+    bh = len(q)
+    s = pu.scale_of(d)
+    runs = []
+    for h in range(bh):
+        qc, ql, qn = eo.kmeans(q[h], qi[h], iters)
+        kc, kl, kn = eo.kmeans(k[h], ki[h], iters)
+        kp, ko = eo.permute(kl, ki.shape[1])
+        runs.append((qc.astype(np.float32), qn.astype(np.int32), kc.astype(np.float32), kl,
+                     kn.astype(np.int32), kp, ko.astype(np.int32)))
+    t = pu.torch_dtype(dtype)
+    qc = np.stack([r[0] for r in runs])
+    qn = np.stack([r[1] for r in runs])
+    kc = np.stack([r[2] for r in runs])
+    kn = np.stack([r[4] for r in runs])
+    kx = np.stack([k[h][runs[h][5]] for h in range(bh)])
+    ko = np.stack([r[6] for r in runs])
+    e = ear.ear_probe(pu.dev(qc), pu.dev(qn), pu.dev(kc), pu.dev(kx, t), pu.dev(ko), s)
+    e_ref = [eo.probe(qc[h], qn[h], k[h], runs[h][3], kc[h], kn[h], s) for h in range(bh)]
+    nq, nk = q.shape[1], k.shape[1]
+    ndiff = 0
+    for mode in (0, 1):
+        for rho in densities:
+            exact, bo, bl, pairs = ear.ear_route(e, pu.dev(qn), pu.dev(kn), nq, nk, rho, mode)
+            exact, bo, bl, pairs = pu.host(exact), pu.host(bo), pu.host(bl), pu.host(pairs)
+            for h in range(bh):
+                ex_ref, p_ref = eo.route(e_ref[h], qn[h], kn[h], nq, nk, rho, mode)
+                nd = pu.assert_route_exact_or_tie(exact[h], ex_ref, e_ref[h], qn[h], kn[h], mode)
+                ndiff += nd
+                if nd == 0:
+                    assert pairs[h] == p_ref
+                o_own, l_own = eo.block_lists(exact[h])
+                np.testing.assert_array_equal(bo[h], o_own)
+                np.testing.assert_array_equal(bl[h][:o_own[-1]], l_own)
+                cost = (qn[h][:, None].astype(np.int64) * kn[h][None, :])[exact[h].astype(bool)]
+                assert pairs[h] == cost.sum() <= math.floor(rho * float(nq * nk))
+    return ndiff
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_probe_then_route_given_oracle_clustering(layers, cfg):
+    L = layers[cfg]
+    w = L.workload
+    _probe_route_case(L.q, L.k, L.q_init, L.k_init, w.iters, w.d,
+                      (0.0, 0.02, 0.05, 0.1, 0.15, 0.25, 0.5, 0.9, 1.0), w.dtype)
+
+
+@pytest.mark.slow
+def test_wan_probe_then_route_given_oracle_clustering():
+    """Two Wan2.x heads (N = 75,600, C_q = 100, C_k = 500): the GPU probe and
+    route from the oracle's clustering reproduce the oracle's routed blocks."""
+    w = gen.WAN
+    L = gen.make_layer(w, heads=[0, w.heads - 1])
+    _probe_route_case(L.q, L.k, L.q_init, L.k_init, w.iters, w.d, (0.05, 0.1, 0.2, 0.4), w.dtype)
+
+
+# --------------------------------------------------------------------------- attention paths
+def _direct_attention(q, k, v, q_sizes, k_sizes, exact, compensate, seed_dtype="bf16"):
+    """Runs ear_attention on hand-built clusters (tokens already grouped by
+    cluster, q_perm = identity) and returns (o, lse, oracle o, oracle lse)."""
+    d = q.shape[1]
+    t = pu.torch_dtype(seed_dtype)
+    qo = np.concatenate([[0], np.cumsum(q_sizes)]).astype(np.int32)
+    ko = np.concatenate([[0], np.cumsum(k_sizes)]).astype(np.int32)
+    ql = np.repeat(np.arange(len(q_sizes)), q_sizes).astype(np.int32)
+    kl = np.repeat(np.arange(len(k_sizes)), k_sizes).astype(np.int32)
+    kc = eo.segment_mean(k, kl, len(k_sizes)).astype(np.float32)
+    vm = eo.segment_mean(v, kl, len(k_sizes)).astype(np.float32)
+    o_lists, l_lists = eo.block_lists(exact)
+    bl = np.zeros(exact.size, np.int32)
+    bl[:len(l_lists)] = l_lists
+    s = pu.scale_of(d)
+    o, lse = ear.ear_attention(
+        pu.dev(q[None], t), pu.dev(k[None], t), pu.dev(v[None], t), pu.dev(qo[None]),
+        pu.dev(ko[None]), pu.dev(np.arange(len(q), dtype=np.int32)[None]), pu.dev(kc[None]),
+        pu.dev(vm[None]), pu.dev(exact[None].astype(np.uint8)), pu.dev(o_lists[None].astype(np.int32)),
+        pu.dev(bl[None]), s, compensate, want_lse=True)
+    o_ref, lse_ref = eo.attention(q, k, v, ql, kl, kc, vm, np.asarray(k_sizes, np.int64),
+                                  exact.astype(np.uint8), s, compensate)
+    return pu.host(o)[0], pu.host(lse)[0], o_ref, lse_ref
+
+
+@pytest.mark.parametrize("pattern", ["all_exact", "mixed"])
+def test_attention_running_max_rescale_path(pattern):
+    """Every later key cluster raises the logits by about 9.8 in base 2, more
+    than the kernel's 2^8 rescale threshold, so the running max moves and O is
+    rescaled in tensor memory on almost every chunk (and on centroid chunks in
+    the mixed case)."""
+    rng = np.random.default_rng(77)
+    d = 128
+    q_sizes = [300]
+    k_sizes = [40, 64, 70, 33, 64, 50]
+    q = gen.round_to_bf16(0.5 * rng.standard_normal((300, d)) + 1.0)
+    shift = np.repeat(0.6 * np.arange(len(k_sizes)), k_sizes)[:, None]
+    k = gen.round_to_bf16(0.5 * rng.standard_normal((sum(k_sizes), d)) + shift)
+    v = gen.round_to_bf16(rng.standard_normal((sum(k_sizes), d)))
+    exact = np.ones((1, len(k_sizes)), np.uint8)
+    if pattern == "mixed":
+        exact[0, [2, 4]] = 0
+    o, lse, o_ref, lse_ref = _direct_attention(q, k, v, q_sizes, k_sizes, exact, True)
+    pu.assert_attention_close(o, o_ref, "bf16")
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=pu.LSE_TOL["bf16"])
+
+
+@pytest.mark.parametrize("compensate", [True, False])
+def test_attention_block_lists_beyond_shared_memory(compensate):
+    """C_k = 2,100 key clusters of 1-3 keys: the unit's block list and the
+    slice's key offsets exceed the 2,048 entries staged in shared memory, so
+    the kernel walks them in global memory."""
+    rng = np.random.default_rng(91)
+    d = 64
+    q_sizes = [130, 70]
+    k_sizes = rng.integers(1, 4, 2100)
+    q = gen.round_to_bf16(rng.standard_normal((sum(q_sizes), d)))
+    k = gen.round_to_bf16(rng.standard_normal((int(k_sizes.sum()), d)))
+    v = gen.round_to_bf16(rng.standard_normal((int(k_sizes.sum()), d)))
+    exact = np.zeros((2, len(k_sizes)), np.uint8)
+    exact[0] = 1                                   # 2,100 listed clusters
+    exact[1] = rng.integers(0, 2, len(k_sizes))    # about half
+    o, lse, o_ref, lse_ref = _direct_attention(q, k, v, q_sizes, k_sizes, exact, compensate)
+    pu.assert_attention_close(o, o_ref, "bf16")
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=pu.LSE_TOL["bf16"])
+
+
+def test_compensated_logits_keep_fp32_centroids(layers, oracle_runs):
+    """At density 0 every term is compensated, so lse = log sum_b |b| e^{s q·k̄_b}
+    isolates the centroid logits: with k̄ as a bf16 hi + lo pair they stay
+    within 1e-4 of the oracle's fp64 values (one bf16 copy would be ~2e-3 off)."""
+    L, runs = layers["mid"], oracle_runs["mid"]
+    w = L.workload
+    none = np.zeros_like(_stack(runs, "exact"))
+    lists = (np.zeros((len(runs), w.c_q + 1), np.int32), np.zeros((len(runs), w.c_q * w.c_k), np.int32))
+    o, lse = _run_attention(L, runs, True, exact=none, lists=lists)
+    worst = 0.0
+    for h, r in enumerate(runs):
+        o_ref, lse_ref = eo.attention(L.q[h], L.k[h], L.v[h], r.q_labels, r.k_labels,
+                                      r.k_cent.astype(np.float32), r.v_mean.astype(np.float32),
+                                      r.k_counts, none[h], pu.scale_of(w.d), True)
+        worst = max(worst, float(np.abs(lse[h] - lse_ref).max()))
+        pu.assert_attention_close(o[h], o_ref, "bf16")
+    print(f"compensated lse max-abs error vs fp64: {worst:.3e}")
+    assert worst <= 1e-4

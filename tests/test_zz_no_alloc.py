@@ -71,3 +71,31 @@ def test_static_permute_rejects_a_problem_larger_than_its_array():
     assert status == N.EAR_ERR_WORKSPACE
     need = N.workspace_bytes(N.EAR_OP_PERMUTE, 40, 75600, 0, 128, 500, 0)
     assert need <= N.PERMUTE_STATIC_MAX_BYTES
+
+
+def test_static_permute_allocates_no_device_memory():
+    """The entry point's defining property: with its outputs already allocated,
+    a Wan-sized call (40 slices x 75,600 tokens in 500 clusters, which needs
+    about 6 MB of scratch) leaves the device's free memory unchanged."""
+    rng = np.random.default_rng(7)
+    bh, n, c, d = 40, 75600, 500, 128
+    lab = torch.from_numpy(rng.integers(0, c, (bh, n)).astype(np.int32)).cuda()
+    x = torch.randn((bh, n, d), device="cuda").to(torch.bfloat16)
+    _static_via_abi(lab, c, x, True)  # first call on this device: loads the module
+    torch.cuda.synchronize()
+    perm = torch.empty((bh, n), dtype=torch.int32, device="cuda")
+    off = torch.empty((bh, c + 1), dtype=torch.int32, device="cuda")
+    xp = torch.empty_like(x)
+    mean = torch.empty((bh, c, d), dtype=torch.float32, device="cuda")
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(2):
+        status = N.lib().ear_permute_static(
+            vp(lab), bh, n, c, vp(perm), vp(off), vp(x), vp(xp), N.EAR_BF16, d, vp(mean),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert status == N.EAR_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    assert ear.ear_get_device_status() == 0
