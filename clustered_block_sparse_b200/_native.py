@@ -13,11 +13,15 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libear.so")
 EAR_OK, EAR_ERR_ARG, EAR_ERR_UNSUPPORTED, EAR_ERR_WORKSPACE, EAR_ERR_CUDA, EAR_ERR_TIMEOUT, \
     EAR_ERR_DEVICE = range(7)
 EAR_F32, EAR_BF16 = 0, 1
-EAR_OP_KMEANS, EAR_OP_PERMUTE, EAR_OP_PROBE, EAR_OP_ROUTE, EAR_OP_ATTENTION = range(5)
+EAR_OP_KMEANS, EAR_OP_PERMUTE, EAR_OP_PROBE, EAR_OP_ROUTE, EAR_OP_ATTENTION, \
+    EAR_OP_ROUTE_ROWS = range(6)
 EAR_COMPENSATE = 1
+EAR_PROBE_LOGIT, EAR_PROBE_WEIGHTS, EAR_PROBE_VALUE = 0, 1, 2
 
 EXPORTED = ("ear_status_string", "ear_workspace_bytes", "ear_kmeans", "ear_permute",
             "ear_permute_apply", "ear_permute_static", "ear_probe", "ear_route", "ear_attention",
+            "ear_route_rows", "ear_topp_budget", "ear_uniform_budget", "ear_cluster_stats",
+            "ear_normalizer_change",
             "ear_get_device_status", "ear_launch_count")
 PERMUTE_STATIC_MAX_BYTES = 8 << 20
 
@@ -55,9 +59,17 @@ def lib() -> ctypes.CDLL:
     L.ear_permute_static.argtypes = [_vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_int,
                                      _i32, _vp, _vp]
     L.ear_probe.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _vp, _i64, _i64, _i32, _i32, _i32,
-                            ctypes.c_float, _vp, _vp, ctypes.c_size_t, _vp]
+                            ctypes.c_float, _i32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     L.ear_route.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, ctypes.c_double, _i32,
                             _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.ear_route_rows.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 ctypes.c_size_t, _vp]
+    L.ear_topp_budget.argtypes = [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, ctypes.c_float,
+                                  ctypes.c_double, _vp, _vp]
+    L.ear_uniform_budget.argtypes = [_vp, _i64, _i32, _i64, ctypes.c_double, _vp, _vp]
+    L.ear_cluster_stats.argtypes = [_vp, ctypes.c_int, _vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp,
+                                    _vp]
+    L.ear_normalizer_change.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
     L.ear_attention.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, _i64, _i64, _i64, _i32, _i32, _i32, ctypes.c_float, _i32,
                                 _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -66,7 +78,8 @@ def lib() -> ctypes.CDLL:
     L.ear_launch_count.restype = ctypes.c_uint64
     for name in ("ear_workspace_bytes", "ear_kmeans", "ear_permute", "ear_permute_apply",
                  "ear_permute_static",
-                 "ear_probe", "ear_route",
+                 "ear_probe", "ear_route", "ear_route_rows", "ear_topp_budget",
+                 "ear_uniform_budget", "ear_cluster_stats", "ear_normalizer_change",
                  "ear_attention", "ear_get_device_status"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L

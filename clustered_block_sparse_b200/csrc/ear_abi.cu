@@ -76,6 +76,7 @@ ear_status ear_workspace_bytes(ear_op op, int64_t bh, int64_t n_q, int64_t n_k, 
     case EAR_OP_PROBE: *bytes = ear::probe_workspace(bh, n_k, d, c_q, c_k); return EAR_OK;
     case EAR_OP_ROUTE: *bytes = ear::route_workspace(bh, c_q, c_k); return EAR_OK;
     case EAR_OP_ATTENTION: *bytes = ear::attention_workspace(bh, n_q, d, c_q, c_k); return EAR_OK;
+    case EAR_OP_ROUTE_ROWS: *bytes = ear::route_rows_workspace(bh, c_q); return EAR_OK;
   }
   return EAR_ERR_ARG;
 }
@@ -131,19 +132,23 @@ ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_
 ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
                      const float* k_centroids, const void* K_perm, ear_dtype dtype,
                      const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V_perm,
+                     const float* v_centroids, float* E, void* ws, size_t ws_bytes,
+                     void* stream) {
   if (!ok_dtype(dtype) || bh < 1 || n_k < 1 || n_k > kMaxN || c_q < 1 || c_k < 1 ||
-      !std::isfinite(scale))
+      !std::isfinite(scale) || mode < EAR_PROBE_LOGIT || mode > EAR_PROBE_VALUE)
     return EAR_ERR_ARG;
   if (!ok_ptr(q_centroids) || !ok_ptr(q_counts) || !ok_ptr(k_centroids) || !ok_ptr(K_perm) ||
       !ok_ptr(k_offsets) || !ok_ptr(E))
     return EAR_ERR_ARG;
+  if (mode == EAR_PROBE_VALUE && (!ok_ptr(V_perm) || !ok_ptr(v_centroids))) return EAR_ERR_ARG;
   if (!ok_d(d) || c_q > kMaxC || c_k > kMaxC || bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
+  if (mode != EAR_PROBE_LOGIT && dtype != EAR_BF16) return EAR_ERR_UNSUPPORTED;
   EAR_TRY(check_ws(ws, ws_bytes, ear::probe_workspace(bh, n_k, d, c_q, c_k)));
   if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
   return ear::probe_run(q_centroids, q_counts, k_centroids, K_perm, dtype, k_offsets, bh, n_k,
-                        d, c_q, c_k, scale, E, ws, static_cast<cudaStream_t>(stream));
+                        d, c_q, c_k, scale, mode, V_perm, v_centroids, E, ws,
+                        static_cast<cudaStream_t>(stream));
 }
 
 ear_status ear_route(const float* E, const int32_t* q_counts, const int32_t* k_counts,
@@ -169,6 +174,71 @@ ear_status ear_route(const float* E, const int32_t* q_counts, const int32_t* k_c
   return ear::route_run(E, q_counts, k_counts, bh, budget, c_q, c_k, ratio_mode, exact,
                         blk_offsets, blk_list, exact_pairs, ws,
                         static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_route_rows(const float* E, const int32_t* q_counts, const int32_t* k_counts,
+                          int64_t bh, int32_t c_q, int32_t c_k, const int64_t* row_budget,
+                          uint8_t* exact, int32_t* blk_offsets, int32_t* blk_list,
+                          int64_t* exact_pairs, void* ws, size_t ws_bytes, void* stream) {
+  if (bh < 1 || c_q < 1 || c_k < 1) return EAR_ERR_ARG;
+  if (!ok_ptr(E) || !ok_ptr(q_counts) || !ok_ptr(k_counts) || !ok_ptr(row_budget) ||
+      !ok_ptr(exact) || !ok_ptr(blk_offsets) || !ok_ptr(blk_list) || !ok_ptr(exact_pairs))
+    return EAR_ERR_ARG;
+  if (c_q > kMaxC || c_k > ear::kRowsMaxCk || (int64_t)c_q * c_k > kMaxN || bh > kMaxBH)
+    return EAR_ERR_UNSUPPORTED;
+  EAR_TRY(check_ws(ws, ws_bytes, ear::route_rows_workspace(bh, c_q)));
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::route_rows_run(E, q_counts, k_counts, bh, c_q, c_k, row_budget, exact, blk_offsets,
+                             blk_list, exact_pairs, ws, static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_topp_budget(const float* q_centroids, const int32_t* q_counts,
+                           const float* k_centroids, const int32_t* k_counts, int64_t bh,
+                           int32_t d, int32_t c_q, int32_t c_k, float scale, double p,
+                           int64_t* row_budget, void* stream) {
+  if (bh < 1 || c_q < 1 || c_k < 1 || !std::isfinite(scale) || !(p >= 0.0 && p <= 1.0))
+    return EAR_ERR_ARG;
+  if (!ok_ptr(q_centroids) || !ok_ptr(q_counts) || !ok_ptr(k_centroids) || !ok_ptr(k_counts) ||
+      !ok_ptr(row_budget))
+    return EAR_ERR_ARG;
+  if (!ok_d(d) || c_q > kMaxC || c_k > ear::kRowsMaxCk || bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::topp_budget_run(q_centroids, q_counts, k_centroids, k_counts, bh, d, c_q, c_k, scale,
+                              p, row_budget, static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_uniform_budget(const int32_t* q_counts, int64_t bh, int32_t c_q, int64_t n_k,
+                              double density, int64_t* row_budget, void* stream) {
+  if (bh < 1 || c_q < 1 || n_k < 1 || n_k > kMaxN || !(density >= 0.0 && density <= 1.0))
+    return EAR_ERR_ARG;
+  if (!ok_ptr(q_counts) || !ok_ptr(row_budget)) return EAR_ERR_ARG;
+  if (c_q > kMaxC || bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::uniform_budget_run(q_counts, bh, c_q, n_k, density, row_budget,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_cluster_stats(const void* X, ear_dtype dtype, const int32_t* labels,
+                             const float* centroids, int64_t bh, int64_t n, int32_t d, int32_t c,
+                             double* mean_sq_dist, double* max_norm, void* stream) {
+  if (!ok_dtype(dtype) || bh < 1 || n < 1 || n > kMaxN || c < 1) return EAR_ERR_ARG;
+  if (!ok_ptr(X) || !ok_ptr(labels) || !ok_ptr(centroids) || !ok_ptr(mean_sq_dist) ||
+      !ok_ptr(max_norm))
+    return EAR_ERR_ARG;
+  if (!ok_d(d) || c > kMaxC || bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::cluster_stats_run(X, dtype, labels, centroids, bh, n, d, c, mean_sq_dist, max_norm,
+                                static_cast<cudaStream_t>(stream));
+}
+
+ear_status ear_normalizer_change(const float* lse_sparse, const float* lse_dense, int64_t bh,
+                                 int64_t n, double* change, void* stream) {
+  if (bh < 1 || n < 1 || n > kMaxN) return EAR_ERR_ARG;
+  if (!ok_ptr(lse_sparse) || !ok_ptr(lse_dense) || !ok_ptr(change)) return EAR_ERR_ARG;
+  if (bh > kMaxBH) return EAR_ERR_UNSUPPORTED;
+  if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
+  return ear::normalizer_change_run(lse_sparse, lse_dense, bh, n, change,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_perm,

@@ -72,20 +72,42 @@ ear_status permute_apply_run(const int32_t* perm, const int32_t* offsets, int64_
                              float* seg_mean, cudaStream_t s);
 
 size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
-// Tensor-core probe (bf16 keys).
-size_t probe_tc_workspace(int64_t bh, int32_t d, int32_t c_q, int32_t c_k);
+// Tensor-core probe (bf16 keys); mode as in ear_probe.
+size_t probe_tc_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
 ear_status probe_tc_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                         const int32_t* koff, int64_t bh, int64_t n_k, int32_t d, int32_t c_q,
-                        int32_t c_k, float scale, float* E, void* ws, cudaStream_t s);
+                        int32_t c_k, float scale, int32_t mode, const void* V, const float* vc,
+                        float* E, void* ws, cudaStream_t s);
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                      ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws, cudaStream_t s);
+                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V,
+                     const float* vc, float* E, void* ws, cudaStream_t s);
 
 size_t route_workspace(int64_t bh, int32_t c_q, int32_t c_k);
 ear_status route_run(const float* E, const int32_t* qn, const int32_t* kn, int64_t bh,
                      int64_t budget, int32_t c_q, int32_t c_k, int32_t mode, uint8_t* exact,
                      int32_t* blk_off, int32_t* blk_list, int64_t* pairs, void* ws,
                      cudaStream_t s);
+
+// Per-query-cluster routing and budgets (route_rows.cu); C_k <= kRowsMaxCk.
+constexpr int32_t kRowsMaxCk = 8192;
+size_t route_rows_workspace(int64_t bh, int32_t c_q);
+ear_status route_rows_run(const float* E, const int32_t* qn, const int32_t* kn, int64_t bh,
+                          int32_t c_q, int32_t c_k, const int64_t* row_budget, uint8_t* exact,
+                          int32_t* blk_off, int32_t* blk_list, int64_t* pairs, void* ws,
+                          cudaStream_t s);
+ear_status topp_budget_run(const float* qc, const int32_t* qn, const float* kc, const int32_t* kn,
+                           int64_t bh, int32_t d, int32_t c_q, int32_t c_k, float scale, double p,
+                           int64_t* budget, cudaStream_t s);
+ear_status uniform_budget_run(const int32_t* qn, int64_t bh, int32_t c_q, int64_t n_k,
+                              double density, int64_t* budget, cudaStream_t s);
+
+// Diagnostics (diag.cu).
+ear_status cluster_stats_run(const void* X, ear_dtype dt, const int32_t* labels,
+                             const float* cent, int64_t bh, int64_t n, int32_t d, int32_t c,
+                             double* mean_sq, double* max_norm, cudaStream_t s);
+ear_status normalizer_change_run(const float* lse_sparse, const float* lse_dense, int64_t bh,
+                                 int64_t n, double* out, cudaStream_t s);
 
 struct AttnArgs {
   const void* Q;

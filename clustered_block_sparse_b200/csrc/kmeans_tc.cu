@@ -14,28 +14,26 @@
 //                (S = X C^T, fp32, 256-column chunks, two TMEM buffers) and
 //                two epilogue warpgroups scan each chunk (alternate 32-column
 //                groups) twice: pass 1 takes the minimum of
-//                d~_c = ||c||^2 - 2 x.c^, pass 2 collects the columns within
+//                d~_c = ||c||^2 - 2 x.c^, pass 2 collects every column within
 //                the rounding margin of the running minimum.  Each warpgroup
 //                keeps its four best candidates by distance and the smallest
 //                distance it had to drop.  One candidate within the margin of
-//                the row's minimum = a certain label, written here; 2-4 go to
-//                an fp64 decision among them; more (a dropped candidate within
-//                the margin, or a row / centroid without an exact fp16 copy)
-//                go to a full fp64 decision.  Each row's outcome is a byte of
-//                its own (certain / pick with n candidates / full), the
-//                candidates go to per-row slots: plain coalesced stores.
-//   km_resolve   one warp per 32-row window of those bytes: picks (fp64
-//                distances of the 2-4 candidates in the order
+//                the row's minimum = a certain label; 2-4 go to an fp64
+//                decision among them; more (a dropped candidate within the
+//                margin, or a row / centroid without an exact fp16 copy) go
+//                to a full fp64 decision.  Each row's outcome is a
+//                byte of its own (moved / pick with n candidates / full), the
+//                candidates and the old label go to per-row slots: plain
+//                coalesced stores, no list counters.
+//   km_resolve   one warp per 32-row window of those bytes: moves (sums[new]
+//                += x, sums[old] -= x, counts likewise, vector fp32 atomics),
+//                picks (fp64 distances of the 2-4 candidates in the order
 //                sum_k (x_k - c_k)^2, k = 0..d-1, ties to the lowest index;
 //                eight rows per warp) and full decisions (the same over all C
-//                centroids, four per lane at a time).  No atomics.
-//   km_sums      member sums and counts of the final labels, from scratch:
-//                per (row chunk, half of d, slice) a shared-memory copy of the
-//                half-sums filled with shared atomics, written out as one
-//                partial sum per chunk.
-//   km_finalize  centroid = the chunks' partial sums added in chunk order /
-//                count (empty clusters keep theirs), and the fp16 copy /
-//                norms / max norm for the next iteration.
+//                centroids, four per lane at a time), each followed by its
+//                move.  After the first iteration only moved rows cost atomics.
+//   km_finalize  centroid = sum / count (empty clusters keep theirs), and the
+//                fp16 copy / norms / max norm for the next iteration.
 //
 // Rounding bound of the approximate distance d~_c = ||c||^2 - 2 x.c^ (c^ =
 // fp16(c), products exact, fp32 accumulation over d terms, ||c||^2 in fp32):
@@ -95,7 +93,8 @@ struct KLayout {
 };
 
 // per-row outcome byte: bits 0-1 kind, bits 2-4 pick candidate count
-constexpr uint8_t kKindNone = 0;    // certain: km_tc wrote the label
+constexpr uint8_t kKindNone = 0;    // certain, label unchanged
+constexpr uint8_t kKindMove = 1;    // certain, label changed (old label in `from`)
 constexpr uint8_t kKindPick = 2;    // 2-4 candidates in `cand`
 constexpr uint8_t kKindFull = 3;    // fp64 decision over every centroid
 
@@ -107,8 +106,9 @@ struct KmTcParams {
   int32_t* labels;          // [BH*N]
   uint8_t* kind;            // [BH*N] outcome byte
   int4* cand;               // [BH*N] pick candidates
+  int32_t* from;            // [BH*N] old label of a moved row
   int64_t N;
-  int C, C_pad;
+  int C, C_pad, first;
   int c_box;  // rows per centroid TMA box (min(256, C_pad))
   float a_coef, b_coef, s_coef;
 };
@@ -425,10 +425,12 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         }
         full = full || keep == 0 || keep > 4;
         if (valid) {
+          const int old = p.first ? -1 : p.labels[g];
           uint8_t kind = kKindFull;
           if (!full && keep == 1) {
             p.labels[g] = kc[0];
-            kind = kKindNone;
+            kind = kc[0] != old ? kKindMove : kKindNone;
+            if (kind == kKindMove) p.from[g] = old;
           } else if (!full) {
             kind = (uint8_t)(kKindPick | (keep << 2));
             p.cand[g] = make_int4(kc[0], kc[1], kc[2], kc[3]);
@@ -524,6 +526,26 @@ __global__ void km_cprep(const float* __restrict__ cent, __half* __restrict__ ch
            D, c < C);
 }
 
+// sums[to] += x, sums[from] -= x (no old cluster when !has_from) for one row;
+// the `gs` lanes of a group (rank `u`) take 4-value slices.
+template <typename T, int D>
+__device__ __forceinline__ void move_row(const T* __restrict__ x, float* __restrict__ sums,
+                                         int32_t* __restrict__ cnt, int64_t hc_to,
+                                         int64_t hc_from, bool has_from, int u, int gs) {
+  for (int k = u * 4; k < D; k += 4 * gs) {
+    const float4 v = make_float4(Elem<T>::load(x, k), Elem<T>::load(x, k + 1),
+                                 Elem<T>::load(x, k + 2), Elem<T>::load(x, k + 3));
+    atomicAdd(reinterpret_cast<float4*>(sums + hc_to * D + k), v);
+    if (has_from)
+      atomicAdd(reinterpret_cast<float4*>(sums + hc_from * D + k),
+                make_float4(-v.x, -v.y, -v.z, -v.w));
+  }
+  if (u == 0) {
+    atomicAdd(cnt + hc_to, 1);
+    if (has_from) atomicAdd(cnt + hc_from, -1);
+  }
+}
+
 // fp64 squared distance in the oracle's order: sum_k (x_k - c_k)^2, k = 0..D-1,
 // one rounding per operation (no contraction)
 template <typename T, int D>
@@ -549,14 +571,13 @@ __device__ __forceinline__ void argmin_lanes(double& best, int& bidx, int width)
   }
 }
 
-// Labels of the rows km_tc could not certify, decided in fp64: one warp per
-// window of 32 rows.  Picks: eight rows per warp at a time, lane 4r + u takes
-// candidate u of row r; full decisions: a lane carries centroids c, c+32,
-// c+64, c+96 (four independent chains, compared in increasing index order).
+// Resolves every row decided in km_tc: one warp per window of 32 rows.
 template <typename T, int D>
 __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ cent, int64_t N,
-                           int C, int64_t rows, int32_t* __restrict__ labels,
-                           const uint8_t* __restrict__ kind, const int4* __restrict__ cand) {
+                           int C, int64_t rows, int32_t* __restrict__ labels, int first,
+                           const uint8_t* __restrict__ kind, const int4* __restrict__ cand,
+                           const int32_t* __restrict__ from, float* __restrict__ sums,
+                           int32_t* __restrict__ cnt) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -564,6 +585,17 @@ __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ ce
   for (int64_t win = warp; win < nwin; win += nw) {
     const int64_t gl = win * 32 + lane;
     const uint8_t kd = gl < rows ? kind[gl] : kKindNone;
+    // moves of certain rows
+    unsigned m = __ballot_sync(0xffffffffu, (kd & 3) == kKindMove);
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1;
+      const int64_t g = win * 32 + i;
+      const int64_t h = g / N;
+      const int old = from[g];
+      move_row<T, D>(X + g * D, sums, cnt, h * C + labels[g], h * C + old, old >= 0, lane, 32);
+    }
+    // picks: eight rows at a time, lane 4r + u takes candidate u of row r
     unsigned pm = __ballot_sync(0xffffffffu, (kd & 3) == kKindPick);
     while (pm) {
       int myrow = -1;
@@ -572,10 +604,11 @@ __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ ce
         pm &= pm - 1;
         if ((lane >> 2) == r) myrow = i;
       }
-      const int u = lane & 3;
+      const int r = lane >> 2, u = lane & 3;
       const bool live = myrow >= 0;
       const int64_t g = win * 32 + (live ? myrow : 0);
       const int64_t h = g / N;
+      const T* x = X + g * D;
       double best = __longlong_as_double(0x7ff0000000000000ll);
       int bidx = C;
       if (live) {
@@ -583,13 +616,21 @@ __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ ce
         if (u < n) {
           const int4 cc = cand[g];
           const int c = u == 0 ? cc.x : u == 1 ? cc.y : u == 2 ? cc.z : cc.w;
-          best = dist64<T, D>(X + g * D, cent + (h * C + c) * (int64_t)D);
+          best = dist64<T, D>(x, cent + (h * C + c) * (int64_t)D);
           bidx = c;
         }
       }
       argmin_lanes(best, bidx, 4);
+      int old = -1;
+      if (live) old = first ? -1 : labels[g];
+      __syncwarp();
       if (live && u == 0) labels[g] = bidx;
+      if (live && bidx != old)
+        move_row<T, D>(x, sums, cnt, h * C + bidx, h * C + old, old >= 0, u, 4);
+      (void)r;
     }
+    // full fp64 decisions: a lane carries centroids c, c+32, c+64, c+96 (four
+    // independent chains, compared in increasing index order)
     unsigned fm = __ballot_sync(0xffffffffu, (kd & 3) == kKindFull);
     while (fm) {
       const int i = __ffs(fm) - 1;
@@ -622,85 +663,17 @@ __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ ce
         if (c3 < C && d3 < best) { best = d3; bidx = c3; }
       }
       argmin_lanes(best, bidx, 32);
+      const int old = first ? -1 : labels[g];
+      __syncwarp();
       if (lane == 0) labels[g] = bidx;
+      if (bidx != old) move_row<T, D>(x, sums, cnt, h * C + bidx, h * C + old, old >= 0, lane, 32);
     }
   }
 }
 
-// Member sums and counts from this iteration's final labels, from scratch:
-// grid = (row chunk, 64-column half of d, slice).  Each CTA adds its chunk's
-// rows into a shared-memory copy of the half-sums [C][64] (shared atomics; a
-// lane takes 8 columns of one row from one 16-byte load, four rows per warp
-// per load, four loads in flight), then writes its partial sums for
-// km_finalize to add up in chunk order.  A row's columns are rotated by
-// 8 (label & 3) in shared memory, and each lane starts at a different one of
-// its 8 columns, to spread the banks the four rows of a warp hit at once.
-constexpr int kSumThreads = 1024;
-template <int D>
-__global__ void __launch_bounds__(kSumThreads, 1)
-km_sums(const uint16_t* __restrict__ X, const int32_t* __restrict__ labels, int64_t N, int C,
-        int chunks, float* __restrict__ psum, int32_t* __restrict__ pcnt, int* status) {
-  extern __shared__ float ss[];                  // [C][64]
-  int* sc = reinterpret_cast<int*>(ss + C * 64);  // [C]
-  const int chunk = blockIdx.x, half = blockIdx.y;
-  const int64_t h = blockIdx.z;
-  for (int i = threadIdx.x; i < C * 64; i += kSumThreads) ss[i] = 0.f;
-  for (int i = threadIdx.x; i < C; i += kSumThreads) sc[i] = 0;
-  __syncthreads();
-  const int64_t r0 = N * chunk / chunks, r1 = N * (chunk + 1) / chunks;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int rg = lane >> 3, part = lane & 7;
-  constexpr int kWarps = kSumThreads / 32;
-  const uint16_t* xh = X + h * N * D + half * 64 + part * 8;
-  const int32_t* lh = labels + h * N;
-  for (int64_t base = r0 + (int64_t)w * 16; base < r1; base += kWarps * 16) {
-    uint4 v[4];
-    int lab[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t row = base + 4 * u + rg;
-      lab[u] = -1;
-      if (row < r1) {
-        lab[u] = lh[row];
-        v[u] = *reinterpret_cast<const uint4*>(xh + row * D);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = lab[u];
-      if (c < 0) continue;
-      if (c >= C) {
-        latch(status, EAR_ERR_DEVICE);
-        continue;
-      }
-      const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      float* rowp = ss + c * 64;
-      const int rot = 8 * (c & 3);
-#pragma unroll
-      for (int i0 = 0; i0 < 8; ++i0) {
-        const int i = (i0 + part) & 7;
-        const uint32_t wv = i < 2 ? w4[0] : i < 4 ? w4[1] : i < 6 ? w4[2] : w4[3];
-        const float x = __uint_as_float((i & 1) ? (wv & 0xFFFF0000u) : (wv << 16));
-        atomicAdd(rowp + ((part * 8 + i + rot) & 63), x);
-      }
-      if (half == 0 && part == 0) atomicAdd(sc + c, 1);
-    }
-  }
-  __syncthreads();
-  float* out = psum + ((h * chunks + chunk) * (int64_t)C) * D + half * 64;
-  for (int i = threadIdx.x; i < C * 64; i += kSumThreads) {
-    const int c = i >> 6, col = i & 63;
-    out[(int64_t)c * D + col] = ss[c * 64 + ((col + 8 * (c & 3)) & 63)];
-  }
-  if (half == 0)
-    for (int i = threadIdx.x; i < C; i += kSumThreads)
-      pcnt[(h * chunks + chunk) * (int64_t)C + i] = sc[i];
-}
-
-// New centroids = the chunks' partial sums added in chunk order / count (an
-// empty cluster keeps its centroid), then the fp16 / norm copies.
-__global__ void km_finalize(const float* __restrict__ psum, const int32_t* __restrict__ pcnt,
-                            int chunks, float* __restrict__ cent, int32_t* __restrict__ counts,
+// new centroids from the running sums, then the fp16 / norm copies
+__global__ void km_finalize(const float* __restrict__ sums, const int32_t* __restrict__ cnt,
+                            float* __restrict__ cent, int32_t* __restrict__ counts,
                             __half* __restrict__ ch, float* __restrict__ cnorm,
                             float* __restrict__ cmax, int* __restrict__ cbad, int C, int C_pad,
                             int D, int64_t rows) {
@@ -709,15 +682,10 @@ __global__ void km_finalize(const float* __restrict__ psum, const int32_t* __res
   if (warp >= rows) return;  // rows = BH * C
   const int64_t h = warp / C;
   const int c = (int)(warp % C);
-  int n = 0;
-  for (int k = 0; k < chunks; ++k) n += pcnt[(h * chunks + k) * (int64_t)C + c];
+  const int n = cnt[warp];
   float* cr = cent + warp * D;
   if (n > 0)
-    for (int d = lane; d < D; d += 32) {
-      float sum = 0.f;
-      for (int k = 0; k < chunks; ++k) sum += psum[((h * chunks + k) * (int64_t)C + c) * D + d];
-      cr[d] = sum / (float)n;
-    }
+    for (int k = lane; k < D; k += 32) cr[k] = sums[warp * D + k] / (float)n;
   if (lane == 0) counts[warp] = n;
   __syncwarp();
   prep_row(cr, ch + (h * C_pad + c) * D, cnorm + h * C_pad + c, cmax + h, cbad + h, D, true);
@@ -755,10 +723,11 @@ bool make_map_f16(CUtensorMap* map, const void* base, int64_t rows, int d, int b
 }
 
 struct TcWs {
-  float* psum;     // [BH][chunks][C][D] partial member sums
-  int32_t* pcnt;   // [BH][chunks][C]
+  float* sums;
+  int32_t* cnt;
   uint8_t* kind;
   int4* cand;
+  int32_t* from;
   __half* xh;
   float* xnorm;
   __half* ch;
@@ -769,20 +738,13 @@ struct TcWs {
 
 int c_pad_of(int32_t c) { return (int)ceil_div(c, 16) * 16; }
 
-// Row chunks per slice for km_sums: about two CTAs per SM over both halves,
-// at least 1024 rows a chunk.
-int sum_chunks(int64_t bh, int64_t n, int32_t d) {
-  const int64_t want = ceil_div(2 * 148, bh * (d / 64));
-  return (int)std::max<int64_t>(1, std::min<int64_t>(want, n / 1024));
-}
-
 TcWs carve(Carver& cv, int64_t bh, int64_t n, int32_t d, int32_t c) {
   TcWs w;
   const int cp = c_pad_of(c);
-  const int chunks = sum_chunks(bh, n, d);
-  w.psum = cv.take<float>((size_t)bh * chunks * c * d);
-  w.pcnt = cv.take<int32_t>((size_t)bh * chunks * c);
+  w.sums = cv.take<float>((size_t)bh * c * d);
+  w.cnt = cv.take<int32_t>((size_t)bh * c);
   w.cand = cv.take<int4>((size_t)bh * n);
+  w.from = cv.take<int32_t>((size_t)bh * n);
   w.kind = cv.take<uint8_t>((size_t)bh * n);
   w.xh = cv.take<__half>((size_t)bh * n * d);
   w.xnorm = cv.take<float>((size_t)bh * n);
@@ -808,6 +770,8 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
 
   if (cent != init)
     EAR_CUDA(cudaMemcpyAsync(cent, init, sizeof(float) * bh * c * D, cudaMemcpyDeviceToDevice, s));
+  EAR_CUDA(cudaMemsetAsync(w.sums, 0, sizeof(float) * bh * c * D, s));
+  EAR_CUDA(cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * bh * c, s));
   km_xprep<D><<<wgrid, 256, 0, s>>>(X, w.xh, w.xnorm, rows);
   EAR_TRY(after_launch());
   EAR_CUDA(cudaMemsetAsync(w.cmax, 0, sizeof(float) * bh * 2, s));
@@ -828,6 +792,7 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   p.labels = labels;
   p.kind = w.kind;
   p.cand = w.cand;
+  p.from = w.from;
   p.N = n;
   p.C = c;
   p.C_pad = cp;
@@ -842,21 +807,17 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   EAR_CUDA(cudaFuncSetAttribute(km_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
   const dim3 grid((unsigned)ceil_div(ceil_div(n, kTileRows), kTilesPerCta), (unsigned)bh);
   const int64_t crow = bh * (int64_t)c;
-  const int chunks = sum_chunks(bh, n, D);
-  const int sum_smem = c * 64 * (int)sizeof(float) + c * (int)sizeof(int);
-  EAR_CUDA(cudaFuncSetAttribute(km_sums<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sum_smem));
   for (int t = 0; t < iters; ++t) {
+    p.first = t == 0 ? 1 : 0;
     km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
     EAR_TRY(after_launch());
-    km_resolve<uint16_t, D><<<rgrid, 256, 0, s>>>(X, cent, n, c, rows, labels, w.kind, w.cand);
-    EAR_TRY(after_launch());
-    km_sums<D><<<dim3((unsigned)chunks, (unsigned)(D / 64), (unsigned)bh), kSumThreads, sum_smem,
-                 s>>>(X, labels, n, c, chunks, w.psum, w.pcnt, status);
+    km_resolve<uint16_t, D><<<rgrid, 256, 0, s>>>(X, cent, n, c, rows, labels, p.first, w.kind,
+                                                  w.cand, w.from, w.sums, w.cnt);
     EAR_TRY(after_launch());
     EAR_CUDA(cudaMemsetAsync(w.cmax, 0, sizeof(float) * bh * 2, s));
-    km_finalize<<<(unsigned)ceil_div(crow, 8), 256, 0, s>>>(w.psum, w.pcnt, chunks, cent, counts,
-                                                           w.ch, w.cnorm, w.cmax, w.cbad, c, cp,
-                                                           D, crow);
+    km_finalize<<<(unsigned)ceil_div(crow, 8), 256, 0, s>>>(w.sums, w.cnt, cent, counts, w.ch,
+                                                           w.cnorm, w.cmax, w.cbad, c, cp, D,
+                                                           crow);
     EAR_TRY(after_launch());
   }
   return EAR_OK;

@@ -170,15 +170,18 @@ ear_status run_t(const float* qc, const int32_t* qn, const float* kc, const void
 }  // namespace
 
 // bf16 keys run on the tensor cores (probe_tc.cu); fp32 keys here.
-size_t probe_workspace(int64_t bh, int64_t, int32_t d, int32_t c_q, int32_t c_k) {
-  return probe_tc_workspace(bh, d, c_q, c_k);
+size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k) {
+  return probe_tc_workspace(bh, n_k, d, c_q, c_k);
 }
 
+// The weight probes (mode 1, 2) are built for bf16 keys only (the ABI rejects
+// them for fp32 before this point).
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                      ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws, cudaStream_t s) {
+                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V,
+                     const float* vc, float* E, void* ws, cudaStream_t s) {
   if (dt == EAR_BF16)
-    return probe_tc_run(qc, qn, kc, K, koff, bh, n_k, d, c_q, c_k, scale, E, ws, s);
+    return probe_tc_run(qc, qn, kc, K, koff, bh, n_k, d, c_q, c_k, scale, mode, V, vc, E, ws, s);
   return d == 64 ? run_t<float, 64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s)
                  : run_t<float, 128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s);
 }

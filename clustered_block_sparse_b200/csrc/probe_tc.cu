@@ -76,7 +76,20 @@ struct PrParams {
   int64_t nseg;           // BH * mtiles segments of Nk key rows each
   float scale;
   int* status;
+  // weight probes (EAR_PROBE_WEIGHTS / EAR_PROBE_VALUE)
+  uint32_t* zmax;         // [BH][mtiles * kM] largest logit of each centroid row, ordered bits
+  const float2* vst;      // [BH][N_k] per permuted key: (|v_j - v̄_b|^2, (v_j - v̄_b)·v̄_b)
+  const float* vnorm;     // [BH][C_k] |v̄_b|^2
 };
+
+// Monotone map of a float onto uint32 (0 is below every float), for atomicMax.
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
 
 // First cluster b in [0, Ck] with koff[b] >= row (koff is non-decreasing; Ck
 // if none).  Called by a whole warp: each round the 32 lanes test 32 evenly
@@ -134,7 +147,14 @@ __device__ __forceinline__ bool seg_of(const PrParams& p, int64_t seg, int64_t l
   return true;
 }
 
-template <int D>
+// MODE 0: the logit-gap probe.  MODE 1 / 2: the weight / value-aware probes;
+// with g = z_j - z̄_b, t = e^g, δ = t - 1 = expm1(g) and u_j = v_j - v̄_b, the
+// block sum is w̄_b^2 * sum_j δ^2 (MODE 1) or
+// w̄_b^2 * sum_j (t^2 |u_j|^2 + 2 t δ u_j·v̄_b + δ^2 |v̄_b|^2) (MODE 2), since
+// w_j = w̄_b t and |t v_j - v̄_b|^2 = |t u_j + δ v̄_b|^2.  This kernel keeps the
+// sums (no running maximum is needed for them) and each row's largest logit;
+// pr_weigh multiplies by w̄_b^2 = e^{2 (z̄_b - m_a)} once m_a is known.
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 pr_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmK,
       const PrParams p) {
@@ -293,16 +313,34 @@ pr_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorM
       int32_t cend_n = cb + 1 < g.b1 ? koff[cb + 2] : 0;
       float2 nm_n = cb + 1 < g.b1 ? nmu_h[(int64_t)(cb + 1) * apad] : make_float2(0.f, 0.f);
       float acc = 0.f;
+      float zm = -INFINITY;  // largest logit of this row seen here (MODE > 0)
+      const float2* vst_h = MODE == 2 ? p.vst + g.h * p.Nk : nullptr;
+      const float* vn_h = MODE == 2 ? p.vnorm + g.h * p.Ck : nullptr;
+      float vn = MODE == 2 && cb < g.b1 ? vn_h[cb] : 0.f;
+      float vn_n = MODE == 2 && cb + 1 < g.b1 ? vn_h[cb + 1] : 0.f;
       auto flush = [&]() {  // cluster cb is complete
         if (a < p.Cq) Erow[cb] = live_a ? acc : 0.f;
         acc = 0.f;
         ++cb;
         cend = cend_n;
         nm = nm_n;
+        vn = vn_n;
         if (cb + 1 < g.b1) {
           cend_n = koff[cb + 2];
           nm_n = nmu_h[(int64_t)(cb + 1) * apad];
+          if (MODE == 2) vn_n = vn_h[cb + 1];
         }
+      };
+      // one term of the block sum for score value sv (raw S) of key row `row`;
+      // st = (|u|^2, u·v̄) of that key (MODE 2)
+      auto term = [&](float sv, float2 st) {
+        const float gg = fmaf(sv, scale, nm.x) + nm.y;
+        if (MODE == 0) return gg * gg;
+        zm = fmaxf(zm, sv * scale);
+        const float dl = expm1f(gg);
+        if (MODE == 1) return dl * dl;
+        const float tt = dl + 1.f;
+        return fmaf(tt * tt, st.x, fmaf(2.f * tt * dl, st.y, dl * dl * vn));
       };
       for (int i = 0; ok && i < g.ntiles; ++i, ++t) {
         const int buf = (int)(t % kAcc);
@@ -317,24 +355,33 @@ pr_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorM
           tmem_ld_wait();
           const int32_t gr = trow + 32 * gq;
           if (gr >= g.r1) break;
+          // MODE 2: lane l holds key gr + l's statistics, broadcast per column
+          float2 stl = make_float2(0.f, 0.f);
+          if (MODE == 2 && gr + lane < g.r1) stl = vst_h[gr + lane];
           if (gr + 32 <= cend) {  // the whole group lies in cluster cb (warp-uniform)
             float s0 = 0.f, s1 = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              const float g0 = fmaf(__uint_as_float(v[j]), scale, nm.x) + nm.y;
-              const float g1 = fmaf(__uint_as_float(v[j + 1]), scale, nm.x) + nm.y;
-              s0 = fmaf(g0, g0, s0);
-              s1 = fmaf(g1, g1, s1);
+              float2 st0 = make_float2(0.f, 0.f), st1 = st0;
+              if (MODE == 2) {
+                st0 = make_float2(__shfl_sync(0xffffffffu, stl.x, j), __shfl_sync(0xffffffffu, stl.y, j));
+                st1 = make_float2(__shfl_sync(0xffffffffu, stl.x, j + 1),
+                                  __shfl_sync(0xffffffffu, stl.y, j + 1));
+              }
+              s0 += term(__uint_as_float(v[j]), st0);
+              s1 += term(__uint_as_float(v[j + 1]), st1);
             }
             acc += s0 + s1;
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
+              float2 st = make_float2(0.f, 0.f);
+              if (MODE == 2)  // every lane joins the shuffle before any break
+                st = make_float2(__shfl_sync(0xffffffffu, stl.x, j), __shfl_sync(0xffffffffu, stl.y, j));
               const int32_t row = gr + j;
               if (row >= g.r1) break;
               while (row >= cend && cb < g.b1) flush();  // empty clusters flush as 0
-              const float gg = fmaf(__uint_as_float(v[j]), scale, nm.x) + nm.y;
-              acc = fmaf(gg, gg, acc);
+              acc += term(__uint_as_float(v[j]), st);
             }
           }
         }
@@ -343,6 +390,8 @@ pr_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorM
       }
       if (ok)
         while (cb < g.b1) flush();  // the last cluster, then empty trailing clusters
+      if (MODE > 0 && a < p.Cq && zm > -INFINITY)
+        atomicMax(p.zmax + g.h * apad + a, ordered_bits(zm));
     }
   }
 
@@ -423,6 +472,66 @@ pr_mu(const float* __restrict__ qc, const float* __restrict__ kc, int Cq, int Ck
   }
 }
 
+// Weight probes: E[a][b] *= e^{2 (z̄_ab - m_a)}, m_a = the row's largest logit
+// over every key of the slice.  Block = (centroid row a, slice).
+__global__ void pr_weigh(float* __restrict__ E, const float2* __restrict__ nmu,
+                         const uint32_t* __restrict__ zmax, int Cq, int Ck, int apad) {
+  const int a = blockIdx.x;
+  const int64_t h = blockIdx.y;
+  const uint32_t mb = zmax[h * apad + a];
+  const float m = from_ordered(mb);
+  float* row = E + (h * Cq + a) * (int64_t)Ck;
+  for (int b = threadIdx.x; b < Ck; b += blockDim.x) {
+    const float2 nm = nmu[(h * Ck + b) * (int64_t)apad + a];
+    const float zbar = -(nm.x + nm.y);
+    row[b] = mb == 0 ? 0.f : row[b] * expf(2.f * (zbar - m));
+  }
+}
+
+// Per permuted key j of cluster b: (|v_j - v̄_b|^2, (v_j - v̄_b)·v̄_b), and
+// |v̄_b|^2.  Block = (key cluster, slice); a warp per key row, lanes over d.
+template <int D>
+__global__ void pr_vstats(const uint16_t* __restrict__ V, const float* __restrict__ vc,
+                          const int32_t* __restrict__ koff, int64_t Nk, int Ck,
+                          float2* __restrict__ vst, float* __restrict__ vnorm, int* status) {
+  constexpr int kPer = D / 32;
+  const int b = blockIdx.x;
+  const int64_t h = blockIdx.y;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int32_t* oh = koff + h * (int64_t)(Ck + 1);
+  int32_t r0 = oh[b], r1 = oh[b + 1];
+  if (r0 < 0 || r1 < r0 || r1 > Nk) {
+    if (threadIdx.x == 0) latch(status, EAR_ERR_DEVICE);
+    r0 = r1 = 0;
+  }
+  float cb[kPer];
+  float nv = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    cb[i] = vc[(h * Ck + b) * (int64_t)D + lane * kPer + i];
+    nv = fmaf(cb[i], cb[i], nv);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, off);
+  if (threadIdx.x == 0) vnorm[h * Ck + b] = nv;
+  for (int32_t j = r0 + w; j < r1; j += nw) {
+    const uint16_t* row = V + (h * Nk + j) * D + lane * kPer;
+    float uu = 0.f, uv = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const float u = bf16_to_f32(row[i]) - cb[i];
+      uu = fmaf(u, u, uu);
+      uv = fmaf(u, cb[i], uv);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      uu += __shfl_xor_sync(0xffffffffu, uu, off);
+      uv += __shfl_xor_sync(0xffffffffu, uv, off);
+    }
+    if (lane == 0) vst[h * Nk + j] = make_float2(uu, uv);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -460,23 +569,30 @@ int mtiles_of(int32_t c_q) { return (int)ceil_div(c_q, kM); }
 struct PrWs {
   uint16_t* qsplit;
   float2* nmu;
+  uint32_t* zmax;
+  float2* vst;
+  float* vnorm;
 };
 
-PrWs carve(Carver& cv, int64_t bh, int32_t d, int32_t c_q, int32_t c_k) {
+PrWs carve(Carver& cv, int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k) {
   const int mt = mtiles_of(c_q);
   PrWs w;
   w.qsplit = cv.take<uint16_t>((size_t)bh * mt * kParts * kM * d);
   w.nmu = cv.take<float2>((size_t)bh * c_k * mt * kM);
+  w.zmax = cv.take<uint32_t>((size_t)bh * mt * kM);
+  w.vst = cv.take<float2>((size_t)bh * n_k);
+  w.vnorm = cv.take<float>((size_t)bh * c_k);
   return w;
 }
 
-template <int D>
+template <int D, int MODE>
 ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const void* K,
                   const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q, int32_t c_k,
-                  float scale, float* E, void* ws, cudaStream_t s) {
+                  float scale, const void* V, const float* vc, float* E, void* ws,
+                  cudaStream_t s) {
   using L = PLayout<D>;
   Carver cv(ws);
-  PrWs w = carve(cv, bh, D, c_q, c_k);
+  PrWs w = carve(cv, bh, n_k, D, c_q, c_k);
   const int mt = mtiles_of(c_q);
   const int64_t total = bh * mt * kParts * kM * D;
   pr_split<<<(unsigned)ceil_div(total, 256), 256, 0, s>>>(qc, w.qsplit, c_q, mt, D, total);
@@ -506,24 +622,44 @@ ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const voi
   p.nseg = nseg;
   p.scale = scale;
   p.status = device_status_word();
-  EAR_CUDA(cudaFuncSetAttribute(pr_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
-  pr_tc<D><<<grid, kThreads, L::kBytes, s>>>(ma, mk, p);
+  p.zmax = w.zmax;
+  p.vst = w.vst;
+  p.vnorm = w.vnorm;
+  if (MODE > 0) EAR_CUDA(cudaMemsetAsync(w.zmax, 0, sizeof(uint32_t) * bh * mt * kM, s));
+  if (MODE == 2) {
+    pr_vstats<D><<<dim3((unsigned)c_k, (unsigned)bh), 128, 0, s>>>(
+        static_cast<const uint16_t*>(V), vc, koff, n_k, c_k, w.vst, w.vnorm, p.status);
+    EAR_TRY(after_launch());
+  }
+  EAR_CUDA(cudaFuncSetAttribute(pr_tc<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kBytes));
+  pr_tc<D, MODE><<<grid, kThreads, L::kBytes, s>>>(ma, mk, p);
+  EAR_TRY(after_launch());
+  if (MODE > 0) {
+    pr_weigh<<<dim3((unsigned)c_q, (unsigned)bh), 128, 0, s>>>(E, w.nmu, w.zmax, c_q, c_k,
+                                                              mt * kM);
+    EAR_TRY(after_launch());
+  }
   return after_launch();
 }
 
 }  // namespace
 
-size_t probe_tc_workspace(int64_t bh, int32_t d, int32_t c_q, int32_t c_k) {
+size_t probe_tc_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k) {
   Carver cv(nullptr);
-  carve(cv, bh, d, c_q, c_k);
+  carve(cv, bh, n_k, d, c_q, c_k);
   return cv.used;
 }
 
 ear_status probe_tc_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
                         const int32_t* koff, int64_t bh, int64_t n_k, int32_t d, int32_t c_q,
-                        int32_t c_k, float scale, float* E, void* ws, cudaStream_t s) {
-  return d == 64 ? run_tc<64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, ws, s)
-                 : run_tc<128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, ws, s);
+                        int32_t c_k, float scale, int32_t mode, const void* V, const float* vc,
+                        float* E, void* ws, cudaStream_t s) {
+#define EAR_PR(DD, MM) run_tc<DD, MM>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, V, vc, E, ws, s)
+  if (d == 64)
+    return mode == 0 ? EAR_PR(64, 0) : mode == 1 ? EAR_PR(64, 1) : EAR_PR(64, 2);
+  return mode == 0 ? EAR_PR(128, 0) : mode == 1 ? EAR_PR(128, 1) : EAR_PR(128, 2);
+#undef EAR_PR
 }
 
 }  // namespace ear

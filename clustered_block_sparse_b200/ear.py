@@ -134,11 +134,18 @@ def ear_permute_static(labels: torch.Tensor, n_clusters: int, x: Optional[torch.
     return perm, offsets, x_perm, mean
 
 
-def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Optional[float] = None):
-    """E[a,b] = sum_{j in b} (s q̄_a·k_j - s q̄_a·k̄_b)^2 (SVG-EAR §4.2). Returns E [BH,C_q,C_k] f32."""
+def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Optional[float] = None,
+              mode: int = 0, v_perm=None, v_centroids=None):
+    """Per-block compensation-error estimate (SVG-EAR §4.2), E [BH,C_q,C_k] f32.
+
+    mode 0: E[a,b] = sum_{j in b} (s q̄_a·k_j - s q̄_a·k̄_b)^2; mode 1: the same on the
+    unnormalized weights e^{z - m_a}; mode 2: value-aware (needs v_perm, v_centroids)."""
     for t, nm in ((q_centroids, "q_centroids"), (q_counts, "q_counts"), (k_centroids, "k_centroids"),
                   (k_perm, "k_perm"), (k_offsets, "k_offsets")):
         _need(t, nm)
+    if mode == N.EAR_PROBE_VALUE:
+        _need(v_perm, "v_perm")
+        _need(v_centroids, "v_centroids")
     bh, c_q, d = q_centroids.shape
     c_k = k_centroids.shape[1]
     n_k = k_perm.shape[1]
@@ -147,7 +154,8 @@ def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Opti
     ws, nb = _workspace(N.EAR_OP_PROBE, bh, 0, n_k, d, c_q, c_k, k_perm.device)
     N.check("ear_probe", N.lib().ear_probe(
         _p(q_centroids), _p(q_counts), _p(k_centroids), _p(k_perm), _dtype(k_perm), _p(k_offsets),
-        bh, n_k, d, c_q, c_k, ctypes.c_float(s), _p(e), _p(ws), nb, _stream(k_perm.device)))
+        bh, n_k, d, c_q, c_k, ctypes.c_float(s), int(mode), _p(v_perm), _p(v_centroids), _p(e),
+        _p(ws), nb, _stream(k_perm.device)))
     return e
 
 
@@ -168,6 +176,87 @@ def ear_route(e, q_counts, k_counts, n_q: int, n_k: int, density: float, ratio_m
         _p(e), _p(q_counts), _p(k_counts), bh, n_q, n_k, c_q, c_k, ctypes.c_double(density),
         int(ratio_mode), _p(exact), _p(blk_off), _p(blk_list), _p(pairs), _p(ws), nb, _stream(dev)))
     return exact, blk_off, blk_list, pairs
+
+
+def ear_route_rows(e, q_counts, k_counts, row_budget):
+    """Greedy error-to-cost routing inside each query cluster under its own budget
+    (SVG-EAR §5 "Implementation"). row_budget [BH,C_q] int64.
+
+    Returns (exact [BH,C_q,C_k] u8, blk_offsets [BH,C_q+1] i32, blk_list [BH,C_q*C_k] i32,
+    exact_pairs [BH] i64)."""
+    for t, nm in ((e, "E"), (q_counts, "q_counts"), (k_counts, "k_counts"),
+                  (row_budget, "row_budget")):
+        _need(t, nm)
+    bh, c_q, c_k = e.shape
+    dev = e.device
+    exact = torch.empty((bh, c_q, c_k), dtype=torch.uint8, device=dev)
+    blk_off = torch.empty((bh, c_q + 1), dtype=torch.int32, device=dev)
+    blk_list = torch.empty((bh, c_q * c_k), dtype=torch.int32, device=dev)
+    pairs = torch.empty((bh,), dtype=torch.int64, device=dev)
+    ws, nb = _workspace(N.EAR_OP_ROUTE_ROWS, bh, 0, 0, 0, c_q, c_k, dev)
+    N.check("ear_route_rows", N.lib().ear_route_rows(
+        _p(e), _p(q_counts), _p(k_counts), bh, c_q, c_k, _p(row_budget), _p(exact), _p(blk_off),
+        _p(blk_list), _p(pairs), _p(ws), nb, _stream(dev)))
+    return exact, blk_off, blk_list, pairs
+
+
+def ear_topp_budget(q_centroids, q_counts, k_centroids, k_counts, p: float,
+                    scale: Optional[float] = None):
+    """SVG2-style adaptive per-query-cluster budgets from the centroid attention
+    mass (top-p). Returns row_budget [BH,C_q] int64."""
+    for t, nm in ((q_centroids, "q_centroids"), (q_counts, "q_counts"),
+                  (k_centroids, "k_centroids"), (k_counts, "k_counts")):
+        _need(t, nm)
+    bh, c_q, d = q_centroids.shape
+    c_k = k_centroids.shape[1]
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty((bh, c_q), dtype=torch.int64, device=q_centroids.device)
+    N.check("ear_topp_budget", N.lib().ear_topp_budget(
+        _p(q_centroids), _p(q_counts), _p(k_centroids), _p(k_counts), bh, d, c_q, c_k,
+        ctypes.c_float(s), ctypes.c_double(p), _p(out), _stream(q_centroids.device)))
+    return out
+
+
+def ear_uniform_budget(q_counts, n_k: int, density: float):
+    """Each query cluster's share floor(rho |a| N_k) of the global budget. [BH,C_q] int64."""
+    _need(q_counts, "q_counts")
+    bh, c_q = q_counts.shape
+    out = torch.empty((bh, c_q), dtype=torch.int64, device=q_counts.device)
+    N.check("ear_uniform_budget", N.lib().ear_uniform_budget(
+        _p(q_counts), bh, c_q, int(n_k), ctypes.c_double(density), _p(out),
+        _stream(q_counts.device)))
+    return out
+
+
+def ear_cluster_stats(x: torch.Tensor, labels: torch.Tensor, centroids: torch.Tensor):
+    """(δ^2 [BH] f64, max row norm [BH] f64): mean squared row-to-centroid distance
+    and largest row norm (SVG-EAR §4.2 bound residual, §5.3)."""
+    for t, nm in ((x, "x"), (labels, "labels"), (centroids, "centroids")):
+        _need(t, nm)
+    bh, n, d = x.shape
+    c = centroids.shape[1]
+    ms = torch.empty((bh,), dtype=torch.float64, device=x.device)
+    mx = torch.empty((bh,), dtype=torch.float64, device=x.device)
+    N.check("ear_cluster_stats", N.lib().ear_cluster_stats(
+        _p(x), _dtype(x), _p(labels), _p(centroids), bh, n, d, c, _p(ms), _p(mx),
+        _stream(x.device)))
+    return ms, mx
+
+
+def bound_residual(delta_sq, k_max, n_k: int, d: int):
+    """The residual 8 δ_q^2 K_max^2 / (N_k d) of the SVG-EAR §4.2 bound."""
+    return 8.0 * delta_sq * k_max ** 2 / (n_k * d)
+
+
+def ear_normalizer_change(lse_sparse: torch.Tensor, lse_dense: torch.Tensor):
+    """Per slice, mean |e^{lse_sparse - lse_dense} - 1| (SVG-EAR §5.1). [BH] f64."""
+    _need(lse_sparse, "lse_sparse")
+    _need(lse_dense, "lse_dense")
+    bh, n = lse_sparse.shape
+    out = torch.empty((bh,), dtype=torch.float64, device=lse_sparse.device)
+    N.check("ear_normalizer_change", N.lib().ear_normalizer_change(
+        _p(lse_sparse), _p(lse_dense), bh, n, _p(out), _stream(lse_sparse.device)))
+    return out
 
 
 def ear_attention(q_perm_x, k_perm_x, v_perm_x, q_offsets, k_offsets, q_perm, k_centroids,

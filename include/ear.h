@@ -73,7 +73,8 @@ typedef enum {
   EAR_OP_PERMUTE = 1,
   EAR_OP_PROBE = 2,
   EAR_OP_ROUTE = 3,
-  EAR_OP_ATTENTION = 4
+  EAR_OP_ATTENTION = 4,
+  EAR_OP_ROUTE_ROWS = 5
 } ear_op;
 
 /* ear_attention flags */
@@ -88,6 +89,7 @@ EAR_API const char* ear_status_string(ear_status s);
  *   op = EAR_OP_KMEANS:  rows N = n_q, clusters C = c_q   (n_k, c_k ignored)
  *   op = EAR_OP_PERMUTE: rows N = n_q, clusters C = c_q   (n_k, c_k ignored)
  *   op = EAR_OP_PROBE / ROUTE / ATTENTION: all sizes as in those calls.
+ *   op = EAR_OP_ROUTE_ROWS: bh and c_q (the rest ignored).
  * Returns EAR_ERR_ARG for negative sizes or a null `bytes`.
  */
 EAR_API ear_status ear_workspace_bytes(ear_op op, int64_t bh, int64_t n_q, int64_t n_k, int32_t d,
@@ -182,6 +184,11 @@ EAR_API ear_status ear_permute_static(const int32_t* labels, int64_t bh, int64_t
                                       void* X_perm, ear_dtype dtype, int32_t d, float* seg_mean,
                                       void* stream);
 
+/* ear_probe modes */
+#define EAR_PROBE_LOGIT 0  /* logit-space gaps (the spec estimate)               */
+#define EAR_PROBE_WEIGHTS 1 /* gaps of the unnormalized attention weights (§4.2 relaxed) */
+#define EAR_PROBE_VALUE 2  /* value-aware gaps of weight x value (§4.3)                 */
+
 /*
  * Compensation-error probe (SVG-EAR §4.2 "Error estimation"; §1: query
  * centroids stand in for individual queries, O(C_q N_k d) work).
@@ -190,15 +197,24 @@ EAR_API ear_status ear_permute_static(const int32_t* labels, int64_t bh, int64_t
  *   k_centroids [BH][C_k][d] float     k̄_b
  *   K_perm      [BH][N_k][d] dtype     keys in cluster-contiguous order
  *   k_offsets   [BH][C_k+1] int32      cluster b = rows [k_offsets[b], k_offsets[b+1])
- *   E           [BH][C_q][C_k] float out
- *       E[a][b] = sum_{j in b} (scale q̄_a·k_j - scale q̄_a·k̄_b)^2
- *   scale is 1/sqrt(d) for the paper's logits.  Empty key clusters get 0.
+ *   mode        EAR_PROBE_LOGIT / _WEIGHTS / _VALUE (the last two: bf16 keys only)
+ *   V_perm      [BH][N_k][d] dtype     values in the keys' order (EAR_PROBE_VALUE; else NULL)
+ *   v_centroids [BH][C_k][d] float     v̄_b (EAR_PROBE_VALUE; else NULL)
+ *   E           [BH][C_q][C_k] float out, with z_j = scale q̄_a·k_j, z̄_b = scale q̄_a·k̄_b:
+ *     LOGIT:   E[a][b] = sum_{j in b} (z_j - z̄_b)^2
+ *     WEIGHTS: E[a][b] = sum_{j in b} (w_j - w̄_b)^2,   w = e^{z - m_a}
+ *     VALUE:   E[a][b] = sum_{j in b} |w_j v_j - w̄_b v̄_b|^2
+ *   where m_a is the largest z_j over all keys of the slice (the running
+ *   maximum of §4.4 at the end of the stream).  scale is 1/sqrt(d) for the
+ *   paper's logits.  Empty key or query clusters get 0.  fp32 keys support
+ *   EAR_PROBE_LOGIT only (EAR_ERR_UNSUPPORTED otherwise).
  */
 EAR_API ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
                      const float* k_centroids, const void* K_perm, ear_dtype dtype,
                      const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, float* E, void* ws,
-                     size_t ws_bytes, void* stream);
+                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V_perm,
+                     const float* v_centroids, float* E, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /*
  * Greedy error-to-cost routing under a density budget (SVG-EAR §4.2 "Error
@@ -226,6 +242,51 @@ EAR_API ear_status ear_route(const float* E, const int32_t* q_counts, const int3
                      void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Greedy error-to-cost routing inside each query cluster, under that
+ * cluster's own budget (SVG-EAR §5 "Implementation": SVG2 assigns an adaptive
+ * budget to each query cluster and SVG-EAR routes at that granularity).
+ *   E, q_counts, k_counts   as in ear_route
+ *   row_budget [BH][C_q] int64     pairs query cluster a may compute exactly
+ *   exact, blk_offsets, blk_list, exact_pairs   out, as in ear_route
+ * For query cluster a: its blocks with |a||b| > 0 in decreasing E[a][b] / |b|
+ * (fp64; within one query cluster the same order as E / (|a||b|)), ties to
+ * the lower b; |a||b| is added while the total stays <= row_budget[a], and
+ * the walk stops at the first block that does not fit.  C_k <= 8192.
+ */
+EAR_API ear_status ear_route_rows(const float* E, const int32_t* q_counts,
+                                  const int32_t* k_counts, int64_t bh, int32_t c_q, int32_t c_k,
+                                  const int64_t* row_budget, uint8_t* exact,
+                                  int32_t* blk_offsets, int32_t* blk_list, int64_t* exact_pairs,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * SVG2-style adaptive budget of each query cluster from its centroid
+ * attention (the score-based top-p selection of SVG-EAR §3.1 / Fig. 2(c)).
+ *   q_centroids [BH][C_q][d], q_counts [BH][C_q], k_centroids [BH][C_k][d],
+ *   k_counts [BH][C_k]; scale = 1/sqrt(d) for the paper's logits; p in [0, 1]
+ *   row_budget [BH][C_q] int64 out
+ * The mass of key cluster b for query cluster a is |b| e^{scale q̄_a·k̄_b}
+ * (computed in fp64) over non-empty b; sorted by decreasing mass (ties to the
+ * lower b), the smallest prefix whose mass reaches p of the total is the
+ * top-p set, and row_budget[a] = |a| x its key count (0 if |a| = 0).  With
+ * E = that mass x |b|, ear_route_rows under these budgets selects exactly the
+ * top-p sets.  C_k <= 8192.  Takes no workspace.
+ */
+EAR_API ear_status ear_topp_budget(const float* q_centroids, const int32_t* q_counts,
+                                   const float* k_centroids, const int32_t* k_counts, int64_t bh,
+                                   int32_t d, int32_t c_q, int32_t c_k, float scale, double p,
+                                   int64_t* row_budget, void* stream);
+
+/*
+ * Each query cluster's share of a global density budget:
+ * row_budget[a] = floor(density * (|a| * N_k)) (the product exact in int64,
+ * then one double product).  Takes no workspace.
+ */
+EAR_API ear_status ear_uniform_budget(const int32_t* q_counts, int64_t bh, int32_t c_q,
+                                      int64_t n_k, double density, int64_t* row_budget,
+                                      void* stream);
+
+/*
  * Block-sparse attention with linear compensation (SVG-EAR §4.1 routing mask,
  * §4.3 Linear Compensation).  For query i of cluster a one softmax runs over
  *   - exact logits scale q_i·k_j, value v_j, for every key j of every key
@@ -250,6 +311,30 @@ EAR_API ear_status ear_attention(const void* Q_perm, const void* K_perm, const v
                          int64_t n_q, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k,
                          float scale, int32_t flags, void* O, float* lse, void* ws,
                          size_t ws_bytes, void* stream);
+
+/*
+ * Clustering diagnostics (SVG-EAR §4.2: the error bound's residual
+ * 8 δ_q^2 K_max^2 / (N_k d); §5.3 "Effect of clustering").
+ *   X [BH][N][d] dtype, labels [BH][N] int32, centroids [BH][C][d] float
+ *   mean_sq_dist [BH] double out   δ^2 = (1/N) sum_i ||x_i - c_{labels[i]}||^2
+ *   max_norm     [BH] double out   max_i ||x_i|| (K_max when X = K)
+ * Per row in fp32, summed over rows in fp64.  A label outside [0, C) latches
+ * EAR_ERR_DEVICE and that row is skipped.  Takes no workspace.
+ */
+EAR_API ear_status ear_cluster_stats(const void* X, ear_dtype dtype, const int32_t* labels,
+                                     const float* centroids, int64_t bh, int64_t n, int32_t d,
+                                     int32_t c, double* mean_sq_dist, double* max_norm,
+                                     void* stream);
+
+/*
+ * Average relative change of the softmax normalizer (SVG-EAR §5.1): per
+ * slice, the mean over the N queries of |Z_sparse / Z_dense - 1| with
+ * Z = e^{lse} (lse from ear_attention with the routed mask, and with every
+ * block exact); a query whose two lse are equal counts 0.
+ *   lse_sparse, lse_dense [BH][N] float; change [BH] double out
+ */
+EAR_API ear_status ear_normalizer_change(const float* lse_sparse, const float* lse_dense,
+                                         int64_t bh, int64_t n, double* change, void* stream);
 
 /*
  * Synchronizes `stream`, then returns in *out the first device-side error

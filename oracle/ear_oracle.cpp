@@ -163,6 +163,65 @@ void oracle_probe(const double* q_cent, const int64_t* q_counts, const double* K
 }
 
 // ---------------------------------------------------------------------------
+// Step 3, variants: error probes on the unnormalized attention weights
+// (SVG-EAR §4.2 "Relaxed optimization problem": the relaxed objective
+// compares unnormalized attention weights; §4.3: a value-aware estimate that
+// also uses v_j and v̄_j, at the same O(C_q N_k d) cost; §4.4: the streaming
+// kernel subtracts the running maximum of the logits before exponentiating).
+//
+// Reading (the per-entry equations are lost in the extracted pages): for query
+// cluster a, z_j = s q̄_a·k_j, z̄_b = s q̄_a·k̄_b, m_a = max over every key j of
+// the slice of z_j (the running maximum at the end of the stream), w_j =
+// e^{z_j - m_a}, w̄_b = e^{z̄_b - m_a}; for key cluster b
+//   mode 1 (weights):      E[a][b] = sum_{j in b} (w_j - w̄_b)^2
+//   mode 2 (value-aware):  E[a][b] = sum_{j in b} || w_j v_j - w̄_b v̄_b ||^2
+// Blocks with an empty query or key cluster get 0.
+// ---------------------------------------------------------------------------
+void oracle_probe_weights(const double* q_cent, const int64_t* q_counts, const double* K,
+                          const int32_t* k_labels, const double* k_cent,
+                          const int64_t* k_counts, const double* V, const double* v_cent,
+                          int64_t N_k, int32_t d, int32_t C_q, int32_t C_k, double scale,
+                          int32_t mode, double* E) {
+#pragma omp parallel for schedule(dynamic)
+  for (int32_t a = 0; a < C_q; ++a) {
+    double* row = E + (size_t)a * C_k;
+    for (int32_t b = 0; b < C_k; ++b) row[b] = 0.0;
+    if (q_counts[a] == 0) continue;
+    const double* qa = q_cent + (size_t)a * d;
+    std::vector<double> z(N_k), zbar(C_k);
+    double m = -std::numeric_limits<double>::infinity();
+    for (int64_t j = 0; j < N_k; ++j) {
+      double dot = 0.0;
+      for (int32_t k = 0; k < d; ++k) dot += qa[k] * K[j * d + k];
+      z[j] = scale * dot;
+      m = std::max(m, z[j]);
+    }
+    for (int32_t b = 0; b < C_k; ++b) {
+      double dot = 0.0;
+      for (int32_t k = 0; k < d; ++k) dot += qa[k] * k_cent[(size_t)b * d + k];
+      zbar[b] = scale * dot;
+    }
+    for (int64_t j = 0; j < N_k; ++j) {
+      const int32_t b = k_labels[j];
+      const double w = std::exp(z[j] - m), wbar = std::exp(zbar[b] - m);
+      if (mode == 1) {
+        const double g = w - wbar;
+        row[b] += g * g;
+      } else {
+        double sq = 0.0;
+        for (int32_t k = 0; k < d; ++k) {
+          const double g = w * V[j * d + k] - wbar * v_cent[(size_t)b * d + k];
+          sq += g * g;
+        }
+        row[b] += sq;
+      }
+    }
+    for (int32_t b = 0; b < C_k; ++b)
+      if (k_counts[b] == 0) row[b] = 0.0;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Step 4: greedy error-to-cost routing (SVG-EAR §4.2 "Error estimation":
 // blocks are taken for exact attention in decreasing order of
 // sum_{(i,j) in block} eps_ij^2 / (|q_c| |k_c|) until the budget is spent;
@@ -206,6 +265,89 @@ void oracle_route(const double* E, const int64_t* q_counts, const int64_t* k_cou
     exact[it.index] = 1;
   }
   *exact_pairs = used;
+}
+
+// ---------------------------------------------------------------------------
+// Step 4, per query cluster (SVG-EAR §5 "Implementation": SVG2 gives every
+// query cluster an adaptive budget, so the routing runs for each query
+// cluster on its own).
+//
+// oracle_route_rows: for query cluster a with budget row_budget[a] (pairs),
+// its blocks with |a||b| > 0 are walked in decreasing E[a][b] / |b| (within a
+// query cluster this is also the order of E / (|a||b|)), ties to the lower b,
+// adding |a||b| while the total stays <= row_budget[a] and stopping at the
+// first block that does not fit.  pairs[a] receives the pairs taken.
+//
+// oracle_topp_budget (reading of SVG2's top-p budget, the score-based
+// selection of SVG-EAR Fig. 2(c)): the key clusters' centroid attention mass
+// for query cluster a is w_b = |b| e^{s q̄_a·k̄_b - max} over non-empty b;
+// sorted by decreasing w (ties to the lower b), the smallest prefix whose
+// cumulative mass reaches p times the total is the top-p set, and the budget
+// is |a| times the key count of that set (0 for an empty query cluster).
+// ---------------------------------------------------------------------------
+void oracle_route_rows(const double* E, const int64_t* q_counts, const int64_t* k_counts,
+                       int32_t C_q, int32_t C_k, const int64_t* row_budget, uint8_t* exact,
+                       int64_t* pairs) {
+  struct Item { double ratio; int32_t b; int64_t cost; };
+  for (int32_t a = 0; a < C_q; ++a) {
+    std::vector<Item> items;
+    for (int32_t b = 0; b < C_k; ++b) {
+      exact[(size_t)a * C_k + b] = 0;
+      const int64_t cost = q_counts[a] * k_counts[b];
+      if (cost == 0) continue;
+      items.push_back({E[(size_t)a * C_k + b] / (double)k_counts[b], b, cost});
+    }
+    std::sort(items.begin(), items.end(), [](const Item& x, const Item& y) {
+      if (x.ratio != y.ratio) return x.ratio > y.ratio;
+      return x.b < y.b;
+    });
+    int64_t used = 0;
+    for (const Item& it : items) {
+      if (used + it.cost > row_budget[a]) break;
+      used += it.cost;
+      exact[(size_t)a * C_k + it.b] = 1;
+    }
+    pairs[a] = used;
+  }
+}
+
+void oracle_topp_budget(const double* q_cent, const int64_t* q_counts, const double* k_cent,
+                        const int64_t* k_counts, int32_t C_q, int32_t C_k, int32_t d,
+                        double scale, double p, int64_t* budget) {
+  for (int32_t a = 0; a < C_q; ++a) {
+    budget[a] = 0;
+    if (q_counts[a] == 0) continue;
+    std::vector<double> z(C_k, -std::numeric_limits<double>::infinity());
+    double zmax = -std::numeric_limits<double>::infinity();
+    for (int32_t b = 0; b < C_k; ++b) {
+      if (k_counts[b] == 0) continue;
+      double dot = 0.0;
+      for (int32_t k = 0; k < d; ++k) dot += q_cent[(size_t)a * d + k] * k_cent[(size_t)b * d + k];
+      z[b] = scale * dot;
+      zmax = std::max(zmax, z[b]);
+    }
+    std::vector<std::pair<double, int32_t>> w;
+    double total = 0.0;
+    for (int32_t b = 0; b < C_k; ++b) {
+      if (k_counts[b] == 0) continue;
+      const double m = (double)k_counts[b] * std::exp(z[b] - zmax);
+      w.push_back({m, b});
+      total += m;
+    }
+    std::sort(w.begin(), w.end(), [](const std::pair<double, int32_t>& x,
+                                     const std::pair<double, int32_t>& y) {
+      if (x.first != y.first) return x.first > y.first;
+      return x.second < y.second;
+    });
+    double cum = 0.0;
+    int64_t keys = 0;
+    for (const auto& it : w) {
+      if (cum >= p * total) break;  // the prefix already reaches p
+      cum += it.first;
+      keys += k_counts[it.second];
+    }
+    budget[a] = q_counts[a] * keys;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -274,6 +416,45 @@ void oracle_attention(const double* Q, const double* K, const double* V,
       lse[i] = -std::numeric_limits<double>::infinity();
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostics (SVG-EAR §4.2 after "Error estimation": the bound's residual
+// 8 δ_q^2 K_max^2 / (N_k d) grows with the clustering error δ_q^2; §5.3
+// "Effect of clustering": δ_q^2 against the number of query centroids; §5.1:
+// the average relative change of the softmax normalizer).
+//
+// Readings: δ^2 = (1/N) sum_i ||x_i - c_{l_i}||^2, the mean squared distance
+// of the rows to their centroids (the k-means objective over N); K_max =
+// max_j ||k_j||.  The normalizer change of query i is |Z_sparse / Z_dense - 1|
+// with Z = e^{lse}, averaged over the queries.
+// ---------------------------------------------------------------------------
+void oracle_cluster_stats(const double* X, const int32_t* labels, const double* centroids,
+                          int64_t N, int32_t d, double* mean_sq_dist, double* max_norm) {
+  double sum = 0.0, mx = 0.0;
+  for (int64_t i = 0; i < N; ++i) {
+    const double* x = X + i * d;
+    const double* c = centroids + (size_t)labels[i] * d;
+    double dist = 0.0, nrm = 0.0;
+    for (int32_t k = 0; k < d; ++k) {
+      const double diff = x[k] - c[k];
+      dist += diff * diff;
+      nrm += x[k] * x[k];
+    }
+    sum += dist;
+    mx = std::max(mx, std::sqrt(nrm));
+  }
+  *mean_sq_dist = N > 0 ? sum / (double)N : 0.0;
+  *max_norm = mx;
+}
+
+double oracle_normalizer_change(const double* lse_sparse, const double* lse_dense, int64_t N) {
+  double sum = 0.0;
+  for (int64_t i = 0; i < N; ++i) {
+    if (lse_sparse[i] == lse_dense[i]) continue;  // also both -inf: no change
+    sum += std::fabs(std::exp(lse_sparse[i] - lse_dense[i]) - 1.0);
+  }
+  return N > 0 ? sum / (double)N : 0.0;
 }
 
 int32_t oracle_max_threads(void) {

@@ -34,14 +34,28 @@ def lib():
         L.oracle_segment_mean.argtypes = [_f64p, _i32p, _i64, _i32, _i32, _f64p]
         L.oracle_probe.argtypes = [_f64p, _i64p, _f64p, _i32p, _f64p, _i64p, _i64, _i32, _i32,
                                    _i32, ctypes.c_double, _f64p]
+        L.oracle_probe_weights.argtypes = [_f64p, _i64p, _f64p, _i32p, _f64p, _i64p, _f64p,
+                                           _f64p, _i64, _i32, _i32, _i32, ctypes.c_double,
+                                           _i32, _f64p]
         L.oracle_route.argtypes = [_f64p, _i64p, _i64p, _i32, _i32, _i64, _i64, ctypes.c_double,
                                    _i32, _u8p, ctypes.POINTER(ctypes.c_int64)]
         L.oracle_attention.argtypes = [_f64p, _f64p, _f64p, _i32p, _i32p, _f64p, _f64p, _i64p,
                                        _u8p, _i64, _i64, _i32, _i32, _i32, ctypes.c_double,
                                        _i32, _f64p, _f64p]
+        L.oracle_cluster_stats.argtypes = [_f64p, _i32p, _f64p, _i64, _i32,
+                                           ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_double)]
+        L.oracle_cluster_stats.restype = None
+        L.oracle_normalizer_change.argtypes = [_f64p, _f64p, _i64]
+        L.oracle_normalizer_change.restype = ctypes.c_double
+        L.oracle_route_rows.argtypes = [_f64p, _i64p, _i64p, _i32, _i32, _i64p, _u8p, _i64p]
+        L.oracle_route_rows.restype = None
+        L.oracle_topp_budget.argtypes = [_f64p, _i64p, _f64p, _i64p, _i32, _i32, _i32,
+                                         ctypes.c_double, ctypes.c_double, _i64p]
+        L.oracle_topp_budget.restype = None
         L.oracle_max_threads.restype = ctypes.c_int32
         for fn in (L.oracle_kmeans, L.oracle_permute, L.oracle_segment_mean, L.oracle_probe,
-                   L.oracle_route, L.oracle_attention):
+                   L.oracle_probe_weights, L.oracle_route, L.oracle_attention):
             fn.restype = None
         _LIB = L
     return _LIB
@@ -103,6 +117,27 @@ def probe(q_cent, q_counts, k, k_labels, k_cent, k_counts, scale):
     e = np.empty((cq, ck), np.float64)
     lib().oracle_probe(q_cent, _ci64(q_counts), k, _ci32(k_labels), k_cent, _ci64(k_counts),
                        k.shape[0], d, cq, ck, float(scale), e)
+    return e
+
+
+PROBE_LOGIT, PROBE_WEIGHTS, PROBE_VALUE = 0, 1, 2
+
+
+def probe_weights(q_cent, q_counts, k, k_labels, k_cent, k_counts, v, v_cent, scale, mode):
+    """Error probes on the unnormalized attention weights (SVG-EAR §4.2 relaxed
+    problem, §4.3 value-aware estimate, §4.4 running maximum): mode 1 sums
+    (w_j - w̄_b)^2, mode 2 sums ||w_j v_j - w̄_b v̄_b||^2, with w = e^{z - m_a}."""
+    q_cent = _f64(q_cent)
+    k = _f64(k)
+    k_cent = _f64(k_cent)
+    cq, d = q_cent.shape
+    ck = k_cent.shape[0]
+    vv = _f64(v) if v is not None else np.zeros_like(k)
+    vc = _f64(v_cent) if v_cent is not None else np.zeros_like(k_cent)
+    e = np.empty((cq, ck), np.float64)
+    lib().oracle_probe_weights(q_cent, _ci64(q_counts), k, _ci32(k_labels), k_cent,
+                               _ci64(k_counts), vv, vc, k.shape[0], d, cq, ck, float(scale),
+                               int(mode), e)
     return e
 
 
@@ -186,3 +221,56 @@ def pipeline(q, k, v, q_init, k_init, iters, density, mode=0, compensate=True,
     bo, bl = block_lists(exact)
     o, lse = attention(q, k, v, ql, kl, kc, vm, kn, exact, s, compensate)
     return HeadResult(qc, ql, qn, kc, kl, kn, qp, qo, kp, ko, vm, e, exact, pairs, bo, bl, o, lse)
+
+
+def cluster_stats(x, labels, centroids):
+    """(δ^2, K_max): mean squared row-to-centroid distance and largest row norm
+    (SVG-EAR §4.2 bound residual, §5.3 "Effect of clustering")."""
+    x = _f64(x)
+    ms = ctypes.c_double(0.0)
+    mx = ctypes.c_double(0.0)
+    lib().oracle_cluster_stats(x, _ci32(labels), _f64(centroids), x.shape[0], x.shape[1],
+                               ctypes.byref(ms), ctypes.byref(mx))
+    return float(ms.value), float(mx.value)
+
+
+def bound_residual(delta_sq, k_max, n_k, d):
+    """The residual 8 δ_q^2 K_max^2 / (N_k d) of the SVG-EAR §4.2 bound."""
+    return 8.0 * delta_sq * k_max ** 2 / (n_k * d)
+
+
+def normalizer_change(lse_sparse, lse_dense):
+    """Average |Z_sparse / Z_dense - 1| over queries, Z = e^{lse} (SVG-EAR §5.1)."""
+    a = _f64(lse_sparse)
+    b = _f64(lse_dense)
+    return float(lib().oracle_normalizer_change(a, b, a.shape[0]))
+
+
+def route_rows(e, q_counts, k_counts, row_budget):
+    """Greedy error-to-cost routing inside each query cluster under its own
+    budget (SVG-EAR §5 "Implementation"). Returns (exact [C_q, C_k], pairs [C_q])."""
+    e = _f64(e)
+    cq, ck = e.shape
+    exact = np.empty((cq, ck), np.uint8)
+    pairs = np.empty(cq, np.int64)
+    lib().oracle_route_rows(e, _ci64(q_counts), _ci64(k_counts), cq, ck, _ci64(row_budget),
+                            exact, pairs)
+    return exact, pairs
+
+
+def topp_budget(q_cent, q_counts, k_cent, k_counts, scale, p):
+    """Per query cluster: |a| x keys of the smallest set of key clusters, by
+    decreasing centroid attention mass, that reaches fraction p of it."""
+    q_cent = _f64(q_cent)
+    k_cent = _f64(k_cent)
+    cq, d = q_cent.shape
+    out = np.empty(cq, np.int64)
+    lib().oracle_topp_budget(q_cent, _ci64(q_counts), k_cent, _ci64(k_counts), cq,
+                             k_cent.shape[0], d, float(scale), float(p), out)
+    return out
+
+
+def uniform_row_budget(q_counts, n_k, density):
+    """Each query cluster's share of the global budget: floor(rho |a| N_k)."""
+    qn = np.asarray(q_counts, np.int64)
+    return np.floor(density * (qn * int(n_k)).astype(np.float64)).astype(np.int64)

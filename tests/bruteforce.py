@@ -82,3 +82,22 @@ def greedy_route(block_err_sum, q_counts, k_counts, n_q, n_k, density):
         used += cost
         exact[idx // c_k, idx % c_k] = 1
     return exact, used
+
+
+def per_entry_weight_error(q_cent, q_labels, k, k_cent, k_labels, scale, v=None, v_cent=None):
+    """Unnormalized-weight estimates for every (query i, key j), with q̄_i for
+    q_i and each query cluster's weights taken relative to e^{m}, m the largest
+    logit s q̄_i·k_j of its row: (w_ij - w̄_ij)^2, or with values
+    ||w_ij v_j - w̄_ij v̄_j||^2."""
+    qbar = np.asarray(q_cent, np.float64)[q_labels]
+    kbar = np.asarray(k_cent, np.float64)[k_labels]
+    z = scale * qbar @ np.asarray(k, np.float64).T
+    zc = scale * qbar @ kbar.T
+    m = z.max(axis=1, keepdims=True)
+    w, wc = np.exp(z - m), np.exp(zc - m)
+    if v is None:
+        return (w - wc) ** 2
+    vv = np.asarray(v, np.float64)
+    vb = np.asarray(v_cent, np.float64)[k_labels]
+    diff = w[:, :, None] * vv[None, :, :] - wc[:, :, None] * vb[None, :, :]
+    return (diff ** 2).sum(axis=2)

@@ -99,12 +99,16 @@ def test_permute_apply_validation(lib):
 
 def test_probe_validation(lib):
     f = lib.ear_probe
-    assert f(FAKE, FAKE, FAKE, FAKE, 1, FAKE, 1, 100, 128, 4, 4, ctypes.c_float(float("nan")),
-             FAKE, None, 0, None) == N.EAR_ERR_ARG
-    assert f(FAKE, FAKE, FAKE, None, 1, FAKE, 1, 100, 128, 4, 4, ctypes.c_float(0.1),
-             FAKE, None, 0, None) == N.EAR_ERR_ARG
-    assert f(FAKE, FAKE, FAKE, FAKE, 1, FAKE, 1, 100, 32, 4, 4, ctypes.c_float(0.1),
-             FAKE, None, 0, None) == N.EAR_ERR_UNSUPPORTED
+
+    def call(K=FAKE, dtype=1, d=128, scale=0.1, mode=0, V=None, vc=None):
+        return f(FAKE, FAKE, FAKE, K, dtype, FAKE, 1, 100, d, 4, 4, ctypes.c_float(scale), mode, V,
+                 vc, FAKE, None, 0, None)
+    assert call(scale=float("nan")) == N.EAR_ERR_ARG
+    assert call(K=None) == N.EAR_ERR_ARG
+    assert call(d=32) == N.EAR_ERR_UNSUPPORTED
+    assert call(mode=3) == N.EAR_ERR_ARG
+    assert call(mode=N.EAR_PROBE_VALUE) == N.EAR_ERR_ARG          # values missing
+    assert call(mode=N.EAR_PROBE_WEIGHTS, dtype=0) == N.EAR_ERR_UNSUPPORTED  # fp32 keys
 
 
 def test_route_validation(lib):
@@ -131,3 +135,21 @@ def test_attention_validation(lib):
 
 def test_status_query_rejects_null(lib):
     assert lib.ear_get_device_status(None, None) == N.EAR_ERR_ARG
+
+
+def test_route_rows_and_budget_validation(lib):
+    f = lib.ear_route_rows
+    assert f(FAKE, FAKE, FAKE, 1, 4, 9000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+             None) == N.EAR_ERR_UNSUPPORTED                       # C_k above 8192
+    assert f(None, FAKE, FAKE, 1, 4, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+             None) == N.EAR_ERR_ARG
+    assert f(FAKE, FAKE, FAKE, 1, 4, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+             None) == N.EAR_ERR_WORKSPACE
+    g = lib.ear_topp_budget
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 128, 4, 4, ctypes.c_float(0.1), ctypes.c_double(1.5),
+             FAKE, None) == N.EAR_ERR_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 96, 4, 4, ctypes.c_float(0.1), ctypes.c_double(0.5),
+             FAKE, None) == N.EAR_ERR_UNSUPPORTED
+    u = lib.ear_uniform_budget
+    assert u(FAKE, 1, 4, 100, ctypes.c_double(-0.5), FAKE, None) == N.EAR_ERR_ARG
+    assert u(None, 1, 4, 100, ctypes.c_double(0.5), FAKE, None) == N.EAR_ERR_ARG

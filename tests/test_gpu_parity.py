@@ -601,3 +601,176 @@ def test_compensated_logits_keep_fp32_centroids(layers, oracle_runs):
         pu.assert_attention_close(o[h], o_ref, "bf16")
     print(f"compensated lse max-abs error vs fp64: {worst:.3e}")
     assert worst <= 1e-4
+
+
+# --------------------------------------------------------------------------- weight probes
+@pytest.mark.parametrize("mode", [1, 2])
+def test_weight_probes_match_oracle(layers, oracle_runs, mode):
+    """The unnormalized-weight and value-aware probes (SVG-EAR §4.2, §4.3) on
+    the tensor cores, given the oracle's clustering (mid configuration, bf16).
+    The GPU sums fp32 terms (expm1f of the logit gap, then the w̄^2 factor), so
+    E is compared at rtol 1e-4 (about 10^2 fp32 roundings per block); blocks
+    far below the row's largest logit fall under fp32's range and are compared
+    against 1e-7 of the largest E."""
+    L, runs = layers["mid"], oracle_runs["mid"]
+    w = L.workload
+    s = pu.scale_of(w.d)
+    qc = _stack(runs, "q_cent", np.float32)
+    kc = _stack(runs, "k_cent", np.float32)
+    vm = _stack(runs, "v_mean", np.float32)
+    kx = np.stack([L.k[h][r.k_perm] for h, r in enumerate(runs)])
+    vx = np.stack([L.v[h][r.k_perm] for h, r in enumerate(runs)])
+    e = ear.ear_probe(pu.dev(qc), pu.dev(_stack(runs, "q_counts", np.int32)), pu.dev(kc),
+                      pu.dev(kx, torch.bfloat16), pu.dev(_stack(runs, "k_offsets", np.int32)), s,
+                      mode=mode, v_perm=pu.dev(vx, torch.bfloat16), v_centroids=pu.dev(vm))
+    e = pu.host(e)
+    for h, r in enumerate(runs):
+        e_ref = eo.probe_weights(qc[h], r.q_counts, L.k[h], r.k_labels, kc[h], r.k_counts,
+                                 L.v[h], vm[h], s, mode)
+        np.testing.assert_allclose(e[h], e_ref, rtol=1e-4, atol=1e-7 * e_ref.max())
+        # routed on these estimates, the GPU and the oracle pick the same blocks
+        # except at ratios within the comparison's 1e-4
+        for rho in (0.05, 0.15, 0.3):
+            ex, _, _, _ = ear.ear_route(pu.dev(e[h][None]), pu.dev(r.q_counts[None].astype(np.int32)),
+                                        pu.dev(r.k_counts[None].astype(np.int32)), w.n, w.n, rho)
+            ex_ref, _ = eo.route(e_ref, r.q_counts, r.k_counts, w.n, w.n, rho)
+            diff = np.argwhere(pu.host(ex)[0] != ex_ref)
+            if len(diff):
+                rr = pu.route_ratio(e_ref, r.q_counts, r.k_counts, 0)
+                cut = rr[ex_ref.astype(bool)].min()
+                for a, b in diff:
+                    assert abs(rr[a, b] - cut) <= 1e-4 * cut
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_weight_probes_vanish_on_constant_clusters(mode):
+    """P2 on the GPU: keys and values equal to their cluster means give E = 0 up
+    to the fp32 logit gap (|g| <~ 1e-4 at d = 128 here), i.e. E <= |b| g^2 (1 + |v̄|^2)
+    ~ 5e-5; a non-constant block is O(1) or larger."""
+    rng = np.random.default_rng(21)
+    d, ck, per, cq = 128, 7, 40, 5
+    kc = gen.round_to_bf16(rng.standard_normal((ck, d)))
+    vc = gen.round_to_bf16(rng.standard_normal((ck, d)))
+    k = np.repeat(kc, per, axis=0)[None]
+    v = np.repeat(vc, per, axis=0)[None]
+    ko = (np.arange(ck + 1) * per).astype(np.int32)[None]
+    qc = rng.standard_normal((1, cq, d)).astype(np.float32)
+    qn = np.full((1, cq), 3, np.int32)
+    e = ear.ear_probe(pu.dev(qc), pu.dev(qn), pu.dev(kc[None]), pu.dev(k, torch.bfloat16),
+                      pu.dev(ko), 0.2, mode=mode, v_perm=pu.dev(v, torch.bfloat16),
+                      v_centroids=pu.dev(vc[None]))
+    assert np.abs(pu.host(e)).max() <= 1e-4
+
+
+# --------------------------------------------------------------------------- per-query-cluster budgets
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+@pytest.mark.parametrize("rho", [0.0, 0.05, 0.15, 0.4, 1.0])
+def test_route_rows_given_same_error_is_bit_exact(oracle_runs, layers, cfg, rho):
+    """Per-query-cluster routing (SVG-EAR §5 "Implementation") under each query
+    cluster's share of the budget: given the oracle's E, the GPU's exact mask,
+    lists and pair count are the oracle's."""
+    runs = oracle_runs[cfg]
+    L = layers[cfg]
+    nk = L.k.shape[1]
+    e = _stack(runs, "e", np.float32)
+    qn = _stack(runs, "q_counts", np.int32)
+    kn = _stack(runs, "k_counts", np.int32)
+    budget = ear.ear_uniform_budget(pu.dev(qn), nk, rho)
+    b_ref = np.stack([eo.uniform_row_budget(qn[h], nk, rho) for h in range(len(runs))])
+    np.testing.assert_array_equal(pu.host(budget), b_ref)
+    exact, bo, bl, pairs = ear.ear_route_rows(pu.dev(e), pu.dev(qn), pu.dev(kn), budget)
+    exact, bo, bl, pairs = pu.host(exact), pu.host(bo), pu.host(bl), pu.host(pairs)
+    for h in range(len(runs)):
+        ex_ref, p_ref = eo.route_rows(e[h].astype(np.float64), qn[h], kn[h], b_ref[h])
+        np.testing.assert_array_equal(exact[h], ex_ref)
+        assert pairs[h] == p_ref.sum()
+        o_ref, l_ref = eo.block_lists(ex_ref)
+        np.testing.assert_array_equal(bo[h], o_ref)
+        np.testing.assert_array_equal(bl[h][:o_ref[-1]], l_ref)
+
+
+@pytest.mark.parametrize("seed", range(2))
+def test_route_rows_ties_empty_clusters_and_budgets(seed):
+    rng = np.random.default_rng(100 + seed)
+    bh, cq, ck = 3, 37, 300
+    qn = rng.integers(0, 40, (bh, cq)).astype(np.int32)
+    kn = rng.integers(0, 25, (bh, ck)).astype(np.int32)
+    qn[:, 2] = 0
+    kn[:, 5] = 0
+    e = (rng.integers(0, 4, (bh, cq, ck)) * kn[:, None, :]).astype(np.float32)  # ratio ties
+    budget = rng.integers(0, 20000, (bh, cq)).astype(np.int64)
+    exact, bo, bl, pairs = ear.ear_route_rows(pu.dev(e), pu.dev(qn), pu.dev(kn), pu.dev(budget))
+    exact, pairs = pu.host(exact), pu.host(pairs)
+    for h in range(bh):
+        ex_ref, p_ref = eo.route_rows(e[h].astype(np.float64), qn[h], kn[h], budget[h])
+        np.testing.assert_array_equal(exact[h], ex_ref)
+        assert pairs[h] == p_ref.sum()
+
+
+@pytest.mark.parametrize("p", [0.3, 0.7, 0.85, 0.95, 1.0])
+def test_topp_budget_matches_oracle(oracle_runs, p):
+    """SVG2-style top-p budgets from the centroid attention mass (fp64 on both
+    sides; a budget may differ only where the oracle's cumulative mass at the
+    cut is within 1e-12 of p times the total)."""
+    runs = oracle_runs["mid"]
+    s = float(np.float32(pu.scale_of(128)))
+    qc = _stack(runs, "q_cent", np.float32)
+    kc = _stack(runs, "k_cent", np.float32)
+    qn = _stack(runs, "q_counts", np.int32)
+    kn = _stack(runs, "k_counts", np.int32)
+    got = pu.host(ear.ear_topp_budget(pu.dev(qc), pu.dev(qn), pu.dev(kc), pu.dev(kn), p, s))
+    for h in range(len(runs)):
+        ref = eo.topp_budget(qc[h], qn[h], kc[h], kn[h], s, p)
+        for a in np.nonzero(got[h] != ref)[0]:
+            live = kn[h] > 0
+            z = s * qc[h][a].astype(np.float64) @ kc[h][live].astype(np.float64).T
+            w = kn[h][live] * np.exp(z - z.max())
+            cum = np.cumsum(np.sort(w)[::-1])
+            assert np.min(np.abs(cum - p * w.sum())) <= 1e-12 * w.sum()
+    # top-p sets: E = mass x |b| routed under these budgets selects exactly them
+    b = ear.ear_topp_budget(pu.dev(qc), pu.dev(qn), pu.dev(kc), pu.dev(kn), p, s)
+    mass = np.zeros((len(runs), qc.shape[1], kc.shape[1]), np.float32)
+    for h in range(len(runs)):
+        z = s * qc[h].astype(np.float64) @ kc[h].astype(np.float64).T
+        m = kn[h][None, :] * np.exp(z - z.max(axis=1, keepdims=True))
+        mass[h] = (m * kn[h][None, :]).astype(np.float32)
+    exact, _, _, pairs = ear.ear_route_rows(pu.dev(mass), pu.dev(qn), pu.dev(kn), b)
+    assert (pu.host(pairs) == pu.host(b).sum(axis=1)).all()
+
+
+# --------------------------------------------------------------------------- diagnostics
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_cluster_stats_match_oracle(layers, oracle_runs, cfg):
+    """δ^2 and K_max (SVG-EAR §4.2 bound residual, §5.3) of the oracle's
+    clustering: rows in fp32, sums in fp64, so rtol 1e-5."""
+    L, runs = layers[cfg], oracle_runs[cfg]
+    w = L.workload
+    t = _tdt(w)
+    for x, lab, cen in ((L.q, "q_labels", "q_cent"), (L.k, "k_labels", "k_cent")):
+        labels = _stack(runs, lab, np.int32)
+        cent = _stack(runs, cen, np.float32)
+        ms, mx = ear.ear_cluster_stats(pu.dev(x, t), pu.dev(labels), pu.dev(cent))
+        ms, mx = pu.host(ms), pu.host(mx)
+        for h in range(len(runs)):
+            ref_ms, ref_mx = eo.cluster_stats(x[h], labels[h], cent[h])
+            np.testing.assert_allclose(ms[h], ref_ms, rtol=1e-5)
+            np.testing.assert_allclose(mx[h], ref_mx, rtol=1e-6)
+        r = ear.bound_residual(ms, mx, x.shape[1], w.d)
+        np.testing.assert_allclose(r, [eo.bound_residual(a, b, x.shape[1], w.d)
+                                       for a, b in zip(ms, mx)], rtol=1e-12)
+
+
+def test_normalizer_change_matches_oracle(layers, oracle_runs):
+    """The SVG-EAR §5.1 statistic from the library's own lse: the routed layer
+    against every block exact (dense), compared with the oracle's formula."""
+    L, runs = layers["mid"], oracle_runs["mid"]
+    full = np.ones_like(_stack(runs, "exact"))
+    lists = (np.stack([eo.block_lists(full[h])[0] for h in range(len(runs))]).astype(np.int32),
+             np.stack([eo.block_lists(full[h])[1] for h in range(len(runs))]).astype(np.int32))
+    _, lse_s = _run_attention(L, runs, True)
+    _, lse_d = _run_attention(L, runs, True, exact=full, lists=lists)
+    got = pu.host(ear.ear_normalizer_change(pu.dev(lse_s), pu.dev(lse_d)))
+    for h in range(len(runs)):
+        ref = eo.normalizer_change(lse_s[h], lse_d[h])
+        np.testing.assert_allclose(got[h], ref, rtol=1e-9)
+    assert np.all(got > 0) and np.all(got < 1)

@@ -300,3 +300,200 @@ def test_pins_catch_a_planted_sign_error():
         wrong[:, b] += (s * qc @ k[j] + s * qc @ kc[b]) ** 2
     e = eo.probe(qc, qn, k, kl, kc, kn, s)
     assert not np.allclose(wrong, e, rtol=1e-6)
+
+
+# --------------------------------------------------------------------------- weight probes
+def _clustered(seed, nq=40, nk=36, d=8, cq=4, ck=5):
+    q, k, v, qi, ki, iters = _head(seed, nq, nk, d, cq, ck)
+    qc, ql, qn = eo.kmeans(q, qi, iters)
+    kc, kl, kn = eo.kmeans(k, ki, iters)
+    vm = eo.segment_mean(v, kl, ck)
+    return q, k, v, qc, ql, qn, kc, kl, kn, vm
+
+
+@pytest.mark.parametrize("seed", range(3))
+@pytest.mark.parametrize("mode", [1, 2])
+def test_weight_probes_match_token_level_bruteforce(seed, mode):
+    """Block sums of the token-level estimates, one row per query: every query of
+    cluster a uses q̄_a, so the block sum is |a| E[a][b] (SVG-EAR §4.2, §4.3)."""
+    q, k, v, qc, ql, qn, kc, kl, kn, vm = _clustered(seed)
+    s = 1 / math.sqrt(q.shape[1])
+    e = eo.probe_weights(qc, qn, k, kl, kc, kn, v, vm, s, mode)
+    per = bf.per_entry_weight_error(qc, ql, k, kc, kl, s, *((v, vm) if mode == 2 else ()))
+    blk = bf.block_sum(per, ql, kl, len(qn), len(kn))
+    ref = blk / np.maximum(qn, 1)[:, None]
+    ref[qn == 0] = 0
+    ref[:, kn == 0] = 0
+    np.testing.assert_allclose(e, ref, rtol=1e-12, atol=1e-300)
+
+
+def test_weight_probes_vanish_on_constant_clusters():
+    """P2: keys and values equal to their cluster means give zero error."""
+    rng = np.random.default_rng(4)
+    d, ck, per = 8, 5, 6
+    kc = rng.standard_normal((ck, d))
+    vc = rng.standard_normal((ck, d))
+    kl = np.repeat(np.arange(ck), per).astype(np.int32)
+    k, v = kc[kl], vc[kl]
+    qc = rng.standard_normal((3, d))
+    qn = np.array([4, 0, 2])
+    kn = np.full(ck, per)
+    for mode in (1, 2):
+        e = eo.probe_weights(qc, qn, k, kl, kc, kn, v, vc, 0.3, mode)
+        assert np.all(e == 0.0)
+
+
+def test_value_aware_probe_with_constant_values_scales_the_weight_probe():
+    """With v_j = v̄_b in every cluster, ||w v̄ - w̄ v̄||^2 = ||v̄||^2 (w - w̄)^2."""
+    q, k, v, qc, ql, qn, kc, kl, kn, vm = _clustered(11)
+    vconst = vm[kl]
+    s = 0.4
+    e1 = eo.probe_weights(qc, qn, k, kl, kc, kn, vconst, vm, s, 1)
+    e2 = eo.probe_weights(qc, qn, k, kl, kc, kn, vconst, vm, s, 2)
+    np.testing.assert_allclose(e2, e1 * (vm ** 2).sum(axis=1)[None, :], rtol=1e-12, atol=1e-300)
+
+
+def test_value_aware_probe_with_constant_keys_is_weighted_value_spread():
+    """With k_j = k̄_b, w_j = w̄_b and the estimate is w̄_b^2 sum_j ||v_j - v̄_b||^2,
+    where w̄_b = e^{s q̄·k̄_b - m}, m the largest logit of the row."""
+    rng = np.random.default_rng(12)
+    d, ck, per = 6, 4, 5
+    kc = rng.standard_normal((ck, d))
+    kl = np.repeat(np.arange(ck), per).astype(np.int32)
+    k = kc[kl]
+    v = rng.standard_normal((ck * per, d))
+    vm = eo.segment_mean(v, kl, ck)
+    qc = rng.standard_normal((3, d))
+    qn = np.ones(3, np.int64)
+    kn = np.full(ck, per)
+    s = 0.5
+    e = eo.probe_weights(qc, qn, k, kl, kc, kn, v, vm, s, 2)
+    zc = s * qc @ kc.T
+    wbar = np.exp(zc - zc.max(axis=1, keepdims=True))
+    spread = np.array([((v[kl == b] - vm[b]) ** 2).sum() for b in range(ck)])
+    np.testing.assert_allclose(e, wbar ** 2 * spread[None, :], rtol=1e-12)
+
+
+def test_weight_probe_small_deviation_limit_is_the_logit_probe():
+    """(e^{z} - e^{z̄})^2 = e^{2 z̄} (z - z̄)^2 (1 + O(z - z̄)): for keys within eta
+    of their centroids the weight probe tends to w̄_b^2 times the logit probe."""
+    rng = np.random.default_rng(13)
+    d, ck, per = 8, 4, 6
+    base = rng.standard_normal((ck, d))
+    kl = np.repeat(np.arange(ck), per).astype(np.int32)
+    qc = rng.standard_normal((2, d))
+    qn = np.array([3, 5])
+    kn = np.full(ck, per)
+    s = 0.35
+    for eta in (1e-3, 1e-4):
+        k = base[kl] + eta * rng.standard_normal((ck * per, d))
+        kc = eo.segment_mean(k, kl, ck)
+        e_w = eo.probe_weights(qc, qn, k, kl, kc, kn, None, None, s, 1)
+        e_l = eo.probe(qc, qn, k, kl, kc, kn, s)
+        z = s * qc @ k.T
+        zc = s * qc @ kc.T
+        wbar2 = np.exp(2 * (zc - z.max(axis=1, keepdims=True)))
+        ratio = e_w / (wbar2 * e_l)
+        assert np.abs(ratio - 1).max() < 50 * eta
+
+
+# --------------------------------------------------------------------------- diagnostics
+def test_cluster_stats_match_numpy_and_the_kmeans_objective():
+    """δ^2 is the k-means objective over N (numpy, written out) and never grows
+    over Lloyd iterations; K_max is the largest row norm."""
+    rng = np.random.default_rng(31)
+    x = _mixture(rng, 300, 16, 7, 0.4)
+    init = x[rng.choice(300, 9, replace=False)]
+    prev = np.inf
+    for it in (1, 2, 4, 8):
+        c, l, _ = eo.kmeans(x, init, it)
+        ds, km = eo.cluster_stats(x, l, c)
+        np.testing.assert_allclose(ds, ((x - c[l]) ** 2).sum(axis=1).mean(), rtol=1e-13)
+        np.testing.assert_allclose(km, np.linalg.norm(x, axis=1).max(), rtol=1e-15)
+        assert ds <= prev * (1 + 1e-12)
+        prev = ds
+    # one centroid per row: zero clustering error
+    ds, _ = eo.cluster_stats(x[:9], np.arange(9), x[:9])
+    assert ds == 0.0
+
+
+def test_bound_residual_and_normalizer_change_closed_forms():
+    assert eo.bound_residual(0.5, 4.0, 1000, 64) == 8 * 0.5 * 16.0 / (1000 * 64)
+    lse = np.array([0.0, 1.0, -2.0])
+    assert eo.normalizer_change(lse, lse) == 0.0
+    # Z doubled for every query: relative change 1; halved: 0.5
+    np.testing.assert_allclose(eo.normalizer_change(lse + math.log(2), lse), 1.0, rtol=1e-15)
+    np.testing.assert_allclose(eo.normalizer_change(lse - math.log(2), lse), 0.5, rtol=1e-15)
+
+
+# --------------------------------------------------------------------------- per-query-cluster budgets
+def _literal_row_greedy(e, qn, kn, budget):
+    exact = np.zeros(e.shape, np.uint8)
+    pairs = np.zeros(e.shape[0], np.int64)
+    for a in range(e.shape[0]):
+        items = sorted(((-e[a, b] / kn[b], b, int(qn[a]) * int(kn[b]))
+                        for b in range(e.shape[1]) if qn[a] * kn[b] > 0))
+        used = 0
+        for _, b, cost in items:
+            if used + cost > budget[a]:
+                break
+            used += cost
+            exact[a, b] = 1
+        pairs[a] = used
+    return exact, pairs
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_route_rows_matches_literal_greedy_per_row(seed):
+    rng = np.random.default_rng(seed)
+    cq, ck = 7, 11
+    qn = rng.integers(0, 6, cq)
+    kn = rng.integers(0, 5, ck)
+    e = rng.integers(0, 4, (cq, ck)).astype(float) * kn[None, :]  # many ratio ties
+    budget = rng.integers(0, 60, cq)
+    exact, pairs = eo.route_rows(e, qn, kn, budget)
+    ref, ref_pairs = _literal_row_greedy(e, qn, kn, budget)
+    np.testing.assert_array_equal(exact, ref)
+    np.testing.assert_array_equal(pairs, ref_pairs)
+    cost = qn[:, None] * kn[None, :]
+    assert np.all((exact * cost).sum(axis=1) == pairs) and np.all(pairs <= budget)
+
+
+def test_route_rows_with_one_row_equals_the_global_route():
+    """With a single query cluster the per-row walk is the global walk of
+    oracle_route under the same budget."""
+    rng = np.random.default_rng(9)
+    qn = np.array([13])
+    kn = rng.integers(0, 9, 30)
+    e = rng.random((1, 30)) * kn[None, :]
+    for rho in (0.0, 0.1, 0.4, 1.0):
+        b = eo.uniform_row_budget(qn, kn.sum(), rho)
+        ex_r, pr = eo.route_rows(e, qn, kn, b)
+        ex_g, pg = eo.route(e, qn, kn, 13, int(kn.sum()), rho)
+        np.testing.assert_array_equal(ex_r, ex_g)
+        assert pr[0] == pg
+
+
+def test_topp_budget_matches_sorted_cumsum_and_special_cases():
+    rng = np.random.default_rng(14)
+    d, cq, ck = 6, 5, 9
+    qc = rng.standard_normal((cq, d))
+    kc = rng.standard_normal((ck, d))
+    qn = np.array([3, 0, 5, 1, 2])
+    kn = np.array([4, 0, 2, 7, 1, 3, 5, 2, 6])
+    s = 0.7
+    for p in (0.01, 0.3, 0.5, 0.85, 0.999999):
+        got = eo.topp_budget(qc, qn, kc, kn, s, p)
+        for a in range(cq):
+            live = kn > 0
+            z = s * qc[a] @ kc[live].T
+            w = kn[live] * np.exp(z - z.max())
+            order = np.lexsort((np.nonzero(live)[0], -w))
+            cum = np.cumsum(w[order]) / w.sum()
+            take = int(np.searchsorted(cum, p - 1e-15) + 1)   # smallest prefix reaching p
+            keys = kn[live][order][:take].sum()
+            assert got[a] == qn[a] * keys
+    # p = 1: every non-empty key cluster; equal masses: ceil(p C) clusters
+    np.testing.assert_array_equal(eo.topp_budget(qc, qn, kc, kn, s, 1.0), qn * kn.sum())
+    flat = eo.topp_budget(np.zeros((1, d)), [1], np.zeros((8, d)), np.ones(8), s, 0.3)
+    assert flat[0] == 3
