@@ -546,6 +546,159 @@ def run_skew_study(args):
     return 0
 
 
+def _study_layer(w, heads, c_q=None):
+    """Cluster, permute and probe one synthetic layer on the GPU (the library's
+    calls); returns the tensors the quality studies route and attend with."""
+    import torch
+
+    from clustered_block_sparse_b200 import ear
+
+    if c_q is not None:
+        w = w.with_(c_q=c_q)
+    layer = gen.make_layer(w, heads=heads)
+    dev = torch.device("cuda", 0)
+    t = torch.bfloat16
+    d = {n: torch.from_numpy(getattr(layer, n)).to(dev, t) for n in ("q", "k", "v")}
+    q_init = torch.from_numpy(layer.q_init).to(dev)  # C_q seeded rows of Q
+    k_init = torch.from_numpy(layer.k_init).to(dev)
+    L = {"w": w, **d}
+    L["qc"], L["ql"], L["qn"] = ear.ear_kmeans(d["q"], q_init, w.iters)
+    L["kc"], L["kl"], L["kn"] = ear.ear_kmeans(d["k"], k_init, w.iters)
+    L["qp"], L["qo"], L["qx"], _ = ear.ear_permute(L["ql"], w.c_q, d["q"])
+    L["kp"], L["ko"], L["kx"], _ = ear.ear_permute(L["kl"], w.c_k, d["k"])
+    L["vx"], L["vm"] = ear.ear_permute_apply(L["kp"], L["ko"], d["v"], seg_mean=True)
+    L["e"] = ear.ear_probe(L["qc"], L["qn"], L["kc"], L["kx"], L["ko"])
+    return L
+
+
+def _sampled_map_errors(L, rows, exact, lse, compensate):
+    """On sampled query rows: the attention-map MSE (1/(N_q N_k)) ||A_sparse -
+    A_full||_F^2 estimated over the sampled rows (SVG-EAR §5.3 "Strategy of block
+    selection"), with A_sparse(i, j) = e^{z_ij - lse_i} on exact blocks,
+    e^{s q_i·k̄_b(j) - lse_i} on compensated ones and 0 on dropped ones (lse from
+    ear_attention); plus the dense normalizer for the same rows.  Plain fp64
+    torch on the GPU: measurement only."""
+    import torch
+
+    w = L["w"]
+    s = 1.0 / math.sqrt(w.d)
+    err2, n_el = 0.0, 0
+    for h, r in enumerate(rows):
+        q = L["q"][h, r].double()
+        k = L["k"][h].double()
+        z = s * q @ k.T                                   # [rows, N_k]
+        full = torch.softmax(z, dim=1)
+        kl = L["kl"][h].long()
+        ql = L["ql"][h, r].long()
+        ex = exact[h][ql][:, kl].bool()                    # token-level mask
+        zc = s * q @ L["kc"][h].double().T                 # [rows, C_k]
+        zs = torch.where(ex, z, zc[:, kl] if compensate else torch.full_like(z, -math.inf))
+        sparse = torch.exp(zs - lse[h, r].double()[:, None])
+        err2 += float(((sparse - full) ** 2).sum())
+        n_el += z.numel()
+    return err2 / n_el
+
+
+def run_fig6a_study(args):
+    """Attention-map MSE against density (SVG-EAR §5.3 "Strategy of block
+    selection", Fig. 6(a)) for top-p selection, top-p with compensation and
+    error-aware routing with compensation, all three under the same SVG2-style
+    per-query-cluster budgets (ear_topp_budget at each p).  Wan-shaped layer,
+    heads 0 and 1, 1024 seeded query rows per head."""
+    import torch
+
+    from clustered_block_sparse_b200 import ear
+
+    w = gen.WAN
+    heads = [0, 1]
+    L = _study_layer(w, heads)
+    s = 1.0 / math.sqrt(w.d)
+    rng = np.random.default_rng(6006)
+    dev = L["q"].device
+    rows = [torch.from_numpy(np.sort(rng.choice(w.n, 1024, replace=False))).to(dev) for _ in heads]
+    knd = L["kn"].double()
+    logw = s * torch.einsum("had,hbd->hab", L["qc"].double(), L["kc"].double())
+    logw = logw + torch.log(knd).unsqueeze(1)
+    mass = torch.softmax(logw, dim=2) * knd.unsqueeze(1)  # E whose E/|b| is the block mass
+    e_score = mass.float().contiguous()
+    table = {}
+    for p in (0.5, 0.7, 0.85, 0.9, 0.95):
+        budget = ear.ear_topp_budget(L["qc"], L["qn"], L["kc"], L["kn"], p)
+        row = {}
+        for name, e, comp in (("topp_dropped", e_score, False), ("topp_compensated", e_score, True),
+                              ("error_routed_compensated", L["e"], True)):
+            exact, bo, bl, pairs = ear.ear_route_rows(e, L["qn"], L["kn"], budget)
+            _, lse = ear.ear_attention(L["qx"], L["kx"], L["vx"], L["qo"], L["ko"], L["qp"],
+                                       L["kc"], L["vm"], exact, bo, bl, compensate=comp,
+                                       want_lse=True)
+            row[name] = _sampled_map_errors(L, rows, exact, lse, comp)
+        row["density"] = float(pairs.double().sum()) / (len(heads) * w.n * w.n)
+        table[f"p={p}"] = row
+    if ear.ear_get_device_status() != 0:
+        raise RuntimeError("device status latched an error in the study")
+    print(json.dumps({"study": "fig6a", "workload": w.name, "heads": heads,
+                      "sampled_query_rows_per_head": 1024,
+                      "metric": "attention-map MSE (1/(N_q N_k)) ||A_sparse - A_full||_F^2",
+                      "budgets": "SVG2-style top-p per query cluster (ear_topp_budget)",
+                      "mse": table}), flush=True)
+    return 0
+
+
+def run_clustering_study(args):
+    """Clustering error and attention error against the number of query
+    centroids (SVG-EAR §5.3 "Effect of clustering", Fig. 6(b)): per C_q, the
+    query clustering error δ_q^2 (ear_cluster_stats), the bound's residual
+    8 δ_q^2 K_max^2 / (N_k d), the attention-map MSE on 1024 sampled rows per
+    head and the average normalizer change against dense attention (§5.1), at
+    top-p budgets with p = 0.85 (the pages' setting, whose density moves with
+    C_q) and at a fixed density 0.10.  Wan-shaped layer, heads 0 and 1."""
+    import torch
+
+    from clustered_block_sparse_b200 import ear
+
+    w = gen.WAN
+    heads = [0, 1]
+    table = {}
+    rng = np.random.default_rng(6007)
+    rows = None
+    for c_q in (25, 50, 100, 200, 300):
+        L = _study_layer(w, heads, c_q=c_q)
+        ww = L["w"]
+        dev = L["q"].device
+        if rows is None:
+            rows = [torch.from_numpy(np.sort(rng.choice(w.n, 1024, replace=False))).to(dev)
+                    for _ in heads]
+        dq, _ = ear.ear_cluster_stats(L["q"], L["ql"], L["qc"])
+        _, kmax = ear.ear_cluster_stats(L["k"], L["kl"], L["kc"])
+        full = torch.ones((len(heads), ww.c_q, ww.c_k), dtype=torch.uint8, device=dev)
+        fo = torch.arange(0, (ww.c_q + 1) * ww.c_k, ww.c_k, device=dev, dtype=torch.int32)
+        fo = fo.unsqueeze(0).expand(len(heads), -1).contiguous()
+        fl = torch.arange(ww.c_k, device=dev, dtype=torch.int32).repeat(ww.c_q)
+        fl = fl.unsqueeze(0).expand(len(heads), -1).contiguous()
+        _, lse_dense = ear.ear_attention(L["qx"], L["kx"], L["vx"], L["qo"], L["ko"], L["qp"],
+                                         L["kc"], L["vm"], full, fo, fl, want_lse=True)
+        entry = {"delta_q_sq": [float(x) for x in dq.cpu()],
+                 "bound_residual": [float(x) for x in
+                                    ear.bound_residual(dq, kmax, w.n, w.d).cpu()]}
+        budgets = (("topp_0.85", ear.ear_topp_budget(L["qc"], L["qn"], L["kc"], L["kn"], 0.85)),
+                   ("density_0.10", ear.ear_uniform_budget(L["qn"], w.n, 0.10)))
+        for name, budget in budgets:
+            exact, bo, bl, pairs = ear.ear_route_rows(L["e"], L["qn"], L["kn"], budget)
+            _, lse = ear.ear_attention(L["qx"], L["kx"], L["vx"], L["qo"], L["ko"], L["qp"],
+                                       L["kc"], L["vm"], exact, bo, bl, want_lse=True)
+            change = ear.ear_normalizer_change(lse, lse_dense)
+            entry[name] = {"attention_map_mse": _sampled_map_errors(L, rows, exact, lse, True),
+                           "normalizer_change": [float(x) for x in change.cpu()],
+                           "density": float(pairs.double().sum()) / (len(heads) * w.n * w.n)}
+        table[f"C_q={c_q}"] = entry
+    if ear.ear_get_device_status() != 0:
+        raise RuntimeError("device status latched an error in the study")
+    print(json.dumps({"study": "clustering", "workload": w.name, "heads": heads,
+                      "budgets": "per query cluster: top-p with p = 0.85, and the share of "
+                                 "density 0.10", "by_c_q": table}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -557,11 +710,15 @@ def main(argv=None):
                     help="override the head count (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--study", choices=("skew",), default=None,
+    ap.add_argument("--study", choices=("skew", "fig6a", "clustering"), default=None,
                     help="run a quality study instead of the timing line")
     args = ap.parse_args(argv)
     if args.study == "skew":
         return run_skew_study(args)
+    if args.study == "fig6a":
+        return run_fig6a_study(args)
+    if args.study == "clustering":
+        return run_clustering_study(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
