@@ -419,87 +419,82 @@ __device__ __forceinline__ void mma_role(const TcParams& p, uint8_t* smem, uint3
   ChunkInfo* info = reinterpret_cast<ChunkInfo*>(smem + L::kInfo);
   {
     {
-      // The whole warp runs this role and computes the operands (so they stay
-      // warp-uniform); one elected lane issues the MMAs and commits.
-      const bool leader = elect_one();
+      // One elected lane runs the whole loop: waits, MMAs and commits.  (A
+      // warp-wide loop with a per-MMA lane predicate was measurably slower.)
       const uint32_t idesc_pv = idesc_bf16(128, D, true);
-      // S of tile t, buffer b: TMEM columns [128 t + 64 b, +64); O_t: [256 + 128 t, +128)
-      // n = keys of the chunk (32 or 64; a centroid chunk is 64: hi rows, then lo rows)
-      auto issue_qk = [&](int t, int buf, int s, int n) {
-        const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
-        const uint64_t qd = desc_sw128(smem_u32(smem + L::kQ + t * L::kTileBytes), 16, 1024);
-        const uint64_t kd = desc_sw128(smem_u32(smem + L::kK + s * L::kStageBytes), 16, 1024);
+      if (elect_one()) {
+        // S of tile t, buffer b: TMEM columns [128 t + 64 b, +64); O_t: [256 + 128 t, +128)
+        // n = keys of the chunk (32 or 64; a centroid chunk is 64: hi rows, then lo rows)
+        auto issue_qk = [&](int t, int buf, int s, int n) {
+          const uint32_t idesc = idesc_bf16(128, (uint32_t)n, false);
+          const uint64_t qd = desc_sw128(smem_u32(smem + L::kQ + t * L::kTileBytes), 16, 1024);
+          const uint64_t kd = desc_sw128(smem_u32(smem + L::kK + s * L::kStageBytes), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = ((kk / 4) * L::kHalfBytes + (kk % 4) * 32) >> 4;
-          const uint32_t ko = ((kk / 4) * L::kSHalf + (kk % 4) * 32) >> 4;
-          if (leader)
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk / 4) * L::kHalfBytes + (kk % 4) * 32) >> 4;
+            const uint32_t ko = ((kk / 4) * L::kSHalf + (kk % 4) * 32) >> 4;
             mma_ss(tmem + kTileRows * t + kChunk * buf, qd + qo, kd + ko, idesc, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, int buf, int s, int n, bool first) {
-        const uint64_t vd = desc_sw128(smem_u32(smem + L::kV + s * L::kStageBytes), L::kSHalf, 1024);
-        const int nk = n / 16;
+          }
+        };
+        auto issue_pv = [&](int t, int buf, int s, int n, bool first) {
+          const uint64_t vd = desc_sw128(smem_u32(smem + L::kV + s * L::kStageBytes), L::kSHalf, 1024);
+          const int nk = n / 16;
 #pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          if (kk < nk && leader)
-            mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kChunk * buf + kk * 8,
-                   vd + ((kk * 2048) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-      };
-      auto commit = [&](uint64_t* bar) {
-        if (leader) mma_commit(bar);
-        __syncwarp();
-      };
-      // n0, n1: keys of chunks c and c+1 (0 = past the end)
-      bool ok = mbar_wait_warp(&bars[kBarQFull], 0, abort) &&
-                mbar_wait_warp(&bars[kBarKvFull], 0, abort);
-      // n0, n1: keys of chunks c and c+1 (0 = past the end)
-      auto keys_of = [&](int st) { return (info[st].comp ? 2 : info[st].nbox) * kBox; };
-      int n0 = ok ? keys_of(0) : 0, n1 = 0;
-      if (ok && n0 > 0) {
-        tc_fence_after();
-        for (int t = 0; t < ntiles; ++t) {
-          issue_qk(t, 0, 0, n0);
-          commit(&bars[kBarSFull + t * kSBufs]);
-        }
-        ok = mbar_wait_warp(&bars[kBarKvFull + 1], 0, abort);
-        n1 = ok ? keys_of(1) : 0;
-        if (ok && n1 > 0) {
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            if (kk < nk)
+              mma_ts(tmem + 256 + kTileRows * t, tmem + kTileRows * t + kChunk * buf + kk * 8,
+                     vd + ((kk * 2048) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+          }
+        };
+        bool ok = mbar_wait(&bars[kBarQFull], 0, abort) && mbar_wait(&bars[kBarKvFull], 0, abort);
+        auto keys_of = [&](int st) { return (info[st].comp ? 2 : info[st].nbox) * kBox; };
+        // n0, n1: keys of chunks c and c+1 (0 = past the end)
+        int n0 = ok ? keys_of(0) : 0, n1 = 0;
+        if (ok && n0 > 0) {
           tc_fence_after();
           for (int t = 0; t < ntiles; ++t) {
-            issue_qk(t, 1, 1, n1);
-            commit(&bars[kBarSFull + t * kSBufs + 1]);
+            issue_qk(t, 0, 0, n0);
+            mma_commit(&bars[kBarSFull + t * kSBufs]);
           }
-        }
-      }
-      for (int c = 0; ok && n0 > 0; ++c) {
-        const int s = c % kStages, buf = c & 1;
-        const int s2 = (c + 2) % kStages;
-        int n2 = 0;
-        for (int t = 0; t < ntiles && ok; ++t) {
-          ok = mbar_wait_warp(&bars[kBarPFull + t * kSBufs + buf], (c >> 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, buf, s, n0, c == 0);
-          commit(&bars[kBarODone + t * kSBufs + buf]);
-          if (t == ntiles - 1) commit(&bars[kBarKvEmpty + s]);
-          if (t == 0 && n1 > 0) {
-            ok = mbar_wait_warp(&bars[kBarKvFull + s2], ((c + 2) / kStages) & 1, abort);
-            if (!ok) break;
-            n2 = keys_of(s2);
+          ok = mbar_wait(&bars[kBarKvFull + 1], 0, abort);
+          n1 = ok ? keys_of(1) : 0;
+          if (ok && n1 > 0) {
             tc_fence_after();
-          }
-          if (n2 > 0) {  // chunk c+2 into the buffer P V of chunk c has just read
-            issue_qk(t, buf, s2, n2);
-            commit(&bars[kBarSFull + t * kSBufs + buf]);
+            for (int t = 0; t < ntiles; ++t) {
+              issue_qk(t, 1, 1, n1);
+              mma_commit(&bars[kBarSFull + t * kSBufs + 1]);
+            }
           }
         }
-        n0 = n1;
-        n1 = n2;
+        for (int c = 0; ok && n0 > 0; ++c) {
+          const int s = c % kStages, buf = c & 1;
+          const int s2 = (c + 2) % kStages;
+          int n2 = 0;
+          for (int t = 0; t < ntiles && ok; ++t) {
+            ok = mbar_wait(&bars[kBarPFull + t * kSBufs + buf], (c >> 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, buf, s, n0, c == 0);
+            mma_commit(&bars[kBarODone + t * kSBufs + buf]);
+            if (t == ntiles - 1) mma_commit(&bars[kBarKvEmpty + s]);
+            if (t == 0 && n1 > 0) {
+              ok = mbar_wait(&bars[kBarKvFull + s2], ((c + 2) / kStages) & 1, abort);
+              if (!ok) break;
+              n2 = keys_of(s2);
+              tc_fence_after();
+            }
+            if (n2 > 0) {  // chunk c+2 into the buffer P V of chunk c has just read
+              issue_qk(t, buf, s2, n2);
+              mma_commit(&bars[kBarSFull + t * kSBufs + buf]);
+            }
+          }
+          n0 = n1;
+          n1 = n2;
+        }
+        // every MMA issued above has finished before TMEM is released
+        mma_commit(&bars[kBarDrain]);
       }
-      // every MMA issued above has finished before TMEM is released
-      commit(&bars[kBarDrain]);
+      __syncwarp();
       mbar_wait_drain(&bars[kBarDrain], 0);
     }
   }
