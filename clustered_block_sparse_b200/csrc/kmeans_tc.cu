@@ -304,11 +304,21 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
     const float cmax = p.cmax[h];
     const bool cbad = p.cbad[h] != 0;
     bool ok = true;
+    // ||x|| and the old label of the next tile's row are loaded a tile ahead
+    auto row_of = [&](int t) { return (tile0 + t) * kTileRows + r; };
+    float xn_next = row_of(0) < p.N ? p.xnorm[h * p.N + row_of(0)] : 0.f;
+    int old_next = (w == 0 && !p.first && row_of(0) < p.N) ? p.labels[h * p.N + row_of(0)] : -1;
     for (int t = 0; t < ntiles; ++t) {
-      const int64_t row = (tile0 + t) * kTileRows + r;
+      const int64_t row = row_of(t);
       const bool valid = row < p.N;
       const int64_t g = h * p.N + row;
-      const float xn = valid ? p.xnorm[g] : 0.f;
+      const float xn = xn_next;
+      const int old_pre = old_next;
+      if (t + 1 < ntiles) {
+        const int64_t rn = row_of(t + 1);
+        xn_next = rn < p.N ? p.xnorm[h * p.N + rn] : 0.f;
+        old_next = (w == 0 && !p.first && rn < p.N) ? p.labels[h * p.N + rn] : -1;
+      }
       const float margin =
           2.f * (p.a_coef * xn * cmax + p.b_coef * cmax * cmax + p.s_coef * (xn + cmax));
       float run = inf;
@@ -425,7 +435,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         }
         full = full || keep == 0 || keep > 4;
         if (valid) {
-          const int old = p.first ? -1 : p.labels[g];
+          const int old = old_pre;
           uint8_t kind = kKindFull;
           if (!full && keep == 1) {
             p.labels[g] = kc[0];
@@ -546,6 +556,13 @@ __device__ __forceinline__ void move_row(const T* __restrict__ x, float* __restr
   }
 }
 
+// four consecutive bf16 values of a row (k a multiple of 4) as one 8-byte load
+__device__ __forceinline__ float4 load4(const uint16_t* x, int k) {
+  const uint2 w = *reinterpret_cast<const uint2*>(x + k);
+  return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+}
+
 // fp64 squared distance in the oracle's order: sum_k (x_k - c_k)^2, k = 0..D-1,
 // one rounding per operation (no contraction)
 template <typename T, int D>
@@ -585,15 +602,45 @@ __global__ void km_resolve(const T* __restrict__ X, const float* __restrict__ ce
   for (int64_t win = warp; win < nwin; win += nw) {
     const int64_t gl = win * 32 + lane;
     const uint8_t kd = gl < rows ? kind[gl] : kKindNone;
-    // moves of certain rows
-    unsigned m = __ballot_sync(0xffffffffu, (kd & 3) == kKindMove);
+    // moves of certain rows: each lane reads its own row's labels, then the
+    // warp moves up to four rows per round with their loads issued together
+    const bool mv = (kd & 3) == kKindMove;
+    int my_to = 0, my_from = -1;
+    if (mv) {
+      my_to = labels[gl];
+      my_from = from[gl];
+    }
+    const int my_h = (int)(gl / N);
+    unsigned m = __ballot_sync(0xffffffffu, mv);
+    const bool part = lane * 4 < D;  // this lane's 4-value slice exists
     while (m) {
-      const int i = __ffs(m) - 1;
-      m &= m - 1;
-      const int64_t g = win * 32 + i;
-      const int64_t h = g / N;
-      const int old = from[g];
-      move_row<T, D>(X + g * D, sums, cnt, h * C + labels[g], h * C + old, old >= 0, lane, 32);
+      int ri[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ri[j] = m ? __ffs(m) - 1 : -1;
+        if (m) m &= m - 1;
+      }
+      float4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (ri[j] >= 0 && part) v[j] = load4(X + (win * 32 + ri[j]) * D, lane * 4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (ri[j] < 0) break;
+        const int64_t hb = (int64_t)__shfl_sync(0xffffffffu, my_h, ri[j]) * C;
+        const int to = __shfl_sync(0xffffffffu, my_to, ri[j]);
+        const int old = __shfl_sync(0xffffffffu, my_from, ri[j]);
+        if (part) {
+          atomicAdd(reinterpret_cast<float4*>(sums + (hb + to) * D + lane * 4), v[j]);
+          if (old >= 0)
+            atomicAdd(reinterpret_cast<float4*>(sums + (hb + old) * D + lane * 4),
+                      make_float4(-v[j].x, -v[j].y, -v[j].z, -v[j].w));
+        }
+        if (lane == 0) {
+          atomicAdd(cnt + hb + to, 1);
+          if (old >= 0) atomicAdd(cnt + hb + old, -1);
+        }
+      }
     }
     // picks: eight rows at a time, lane 4r + u takes candidate u of row r
     unsigned pm = __ballot_sync(0xffffffffu, (kd & 3) == kKindPick);
