@@ -604,12 +604,13 @@ def run_fig6a_study(args):
     selection", Fig. 6(a)) for top-p selection, top-p with compensation and
     error-aware routing with compensation, all three under the same SVG2-style
     per-query-cluster budgets (ear_topp_budget at each p).  Wan-shaped layer,
-    heads 0 and 1, 1024 seeded query rows per head."""
+    heads 0 and 1, 1024 seeded query rows per head, at the pages' Fig. 6(a)
+    setting Q_C = 300, K_C = 1000 unless --c-q / --c-k say otherwise."""
     import torch
 
     from clustered_block_sparse_b200 import ear
 
-    w = gen.WAN
+    w = gen.WAN.with_(c_q=args.c_q or 300, c_k=args.c_k or 1000)
     heads = [0, 1]
     L = _study_layer(w, heads)
     s = 1.0 / math.sqrt(w.d)
@@ -621,12 +622,18 @@ def run_fig6a_study(args):
     logw = logw + torch.log(knd).unsqueeze(1)
     mass = torch.softmax(logw, dim=2) * knd.unsqueeze(1)  # E whose E/|b| is the block mass
     e_score = mass.float().contiguous()
+    # the exp-space and value-aware probes (weight-space errors) beside the logit probe
+    e_w = ear.ear_probe(L["qc"], L["qn"], L["kc"], L["kx"], L["ko"], mode=1)
+    e_v = ear.ear_probe(L["qc"], L["qn"], L["kc"], L["kx"], L["ko"], mode=2, v_perm=L["vx"],
+                        v_centroids=L["vm"])
     table = {}
     for p in (0.5, 0.7, 0.85, 0.9, 0.95):
         budget = ear.ear_topp_budget(L["qc"], L["qn"], L["kc"], L["kn"], p)
         row = {}
         for name, e, comp in (("topp_dropped", e_score, False), ("topp_compensated", e_score, True),
-                              ("error_routed_compensated", L["e"], True)):
+                              ("error_routed_compensated", L["e"], True),
+                              ("weight_error_routed_compensated", e_w, True),
+                              ("value_error_routed_compensated", e_v, True)):
             exact, bo, bl, pairs = ear.ear_route_rows(e, L["qn"], L["kn"], budget)
             _, lse = ear.ear_attention(L["qx"], L["kx"], L["vx"], L["qo"], L["ko"], L["qp"],
                                        L["kc"], L["vm"], exact, bo, bl, compensate=comp,
@@ -637,7 +644,7 @@ def run_fig6a_study(args):
     if ear.ear_get_device_status() != 0:
         raise RuntimeError("device status latched an error in the study")
     print(json.dumps({"study": "fig6a", "workload": w.name, "heads": heads,
-                      "sampled_query_rows_per_head": 1024,
+                      "c_q": w.c_q, "c_k": w.c_k, "sampled_query_rows_per_head": 1024,
                       "metric": "attention-map MSE (1/(N_q N_k)) ||A_sparse - A_full||_F^2",
                       "budgets": "SVG2-style top-p per query cluster (ear_topp_budget)",
                       "mse": table}), flush=True)
@@ -651,12 +658,13 @@ def run_clustering_study(args):
     8 δ_q^2 K_max^2 / (N_k d), the attention-map MSE on 1024 sampled rows per
     head and the average normalizer change against dense attention (§5.1), at
     top-p budgets with p = 0.85 (the pages' setting, whose density moves with
-    C_q) and at a fixed density 0.10.  Wan-shaped layer, heads 0 and 1."""
+    C_q) and at a fixed density 0.10.  Wan-shaped layer, heads 0 and 1, at the
+    pages' Fig. 6(b) setting K_C = 1000 unless --c-k says otherwise."""
     import torch
 
     from clustered_block_sparse_b200 import ear
 
-    w = gen.WAN
+    w = gen.WAN.with_(c_k=args.c_k or 1000)
     heads = [0, 1]
     table = {}
     rng = np.random.default_rng(6007)
@@ -680,10 +688,14 @@ def run_clustering_study(args):
         entry = {"delta_q_sq": [float(x) for x in dq.cpu()],
                  "bound_residual": [float(x) for x in
                                     ear.bound_residual(dq, kmax, w.n, w.d).cpu()]}
-        budgets = (("topp_0.85", ear.ear_topp_budget(L["qc"], L["qn"], L["kc"], L["kn"], 0.85)),
-                   ("density_0.10", ear.ear_uniform_budget(L["qn"], w.n, 0.10)))
-        for name, budget in budgets:
-            exact, bo, bl, pairs = ear.ear_route_rows(L["e"], L["qn"], L["kn"], budget)
+        e_v = ear.ear_probe(L["qc"], L["qn"], L["kc"], L["kx"], L["ko"], mode=2, v_perm=L["vx"],
+                            v_centroids=L["vm"])
+        topp = ear.ear_topp_budget(L["qc"], L["qn"], L["kc"], L["kn"], 0.85)
+        dens = ear.ear_uniform_budget(L["qn"], w.n, 0.10)
+        arms = (("topp_0.85", L["e"], topp), ("density_0.10", L["e"], dens),
+                ("value_topp_0.85", e_v, topp), ("value_density_0.10", e_v, dens))
+        for name, e, budget in arms:
+            exact, bo, bl, pairs = ear.ear_route_rows(e, L["qn"], L["kn"], budget)
             _, lse = ear.ear_attention(L["qx"], L["kx"], L["vx"], L["qo"], L["ko"], L["qp"],
                                        L["kc"], L["vm"], exact, bo, bl, want_lse=True)
             change = ear.ear_normalizer_change(lse, lse_dense)
@@ -693,9 +705,10 @@ def run_clustering_study(args):
         table[f"C_q={c_q}"] = entry
     if ear.ear_get_device_status() != 0:
         raise RuntimeError("device status latched an error in the study")
-    print(json.dumps({"study": "clustering", "workload": w.name, "heads": heads,
+    print(json.dumps({"study": "clustering", "workload": w.name, "heads": heads, "c_k": w.c_k,
                       "budgets": "per query cluster: top-p with p = 0.85, and the share of "
-                                 "density 0.10", "by_c_q": table}), flush=True)
+                                 "density 0.10; routed on the logit probe, and (value_*) on the "
+                                 "value-aware probe", "by_c_q": table}), flush=True)
     return 0
 
 
@@ -712,6 +725,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--study", choices=("skew", "fig6a", "clustering"), default=None,
                     help="run a quality study instead of the timing line")
+    ap.add_argument("--c-q", type=int, default=None, help="query clusters of a study")
+    ap.add_argument("--c-k", type=int, default=None, help="key clusters of a study")
     args = ap.parse_args(argv)
     if args.study == "skew":
         return run_skew_study(args)
