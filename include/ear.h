@@ -185,7 +185,7 @@ EAR_API ear_status ear_permute_static(const int32_t* labels, int64_t bh, int64_t
                                       void* stream);
 
 /* ear_probe modes */
-#define EAR_PROBE_LOGIT 0  /* logit-space gaps (the spec estimate)               */
+#define EAR_PROBE_LOGIT 0  /* logit-space gaps (§4.2 "Error estimation")             */
 #define EAR_PROBE_WEIGHTS 1 /* gaps of the unnormalized attention weights (§4.2 relaxed) */
 #define EAR_PROBE_VALUE 2  /* value-aware gaps of weight x value (§4.3)                 */
 
