@@ -1,6 +1,9 @@
 // Lloyd k-means on the sm_100a tensor cores (SVG-EAR §4.1: Q and K are
 // clustered and each token is represented by the mean token of its cluster).
-// Used for bf16 inputs with C <= 512 centroids; labels are exact.
+// Used for bf16 inputs with C <= 2048 centroids; labels are exact.  Up to 512
+// centroids sit in shared memory at a time: beyond that km_tc runs in passes
+// of 512 centroids, each row's candidate state carried between passes in
+// global memory, and only the last pass decides.
 //
 // Per call:
 //   km_xprep     X (bf16) -> fp16 copy Xh plus ||x|| per row.  A row with a
@@ -62,7 +65,8 @@ using namespace sm100;
 constexpr int kTileRows = 128;
 constexpr int kTilesPerCta = 16;
 constexpr int kColChunk = 256;
-constexpr int kMaxCPad = 512;
+constexpr int kMaxCPad = 512;     // centroids of one km_tc pass
+constexpr int kMaxCTotal = 2048;  // centroids over all passes
 constexpr int kXStages = 2;
 constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 epilogue
 
@@ -110,6 +114,12 @@ struct KmTcParams {
   int64_t N;
   int C, C_pad, first;
   int c_box;  // rows per centroid TMA box (min(256, C_pad))
+  int c0, cp_pass;             // this pass: centroids [c0, c0 + cp_pass) of the padded C_pad
+  int carry_in, carry_out;     // read / write the row state of earlier / later passes
+  float* st_run;               // [BH*N] smallest d~ so far
+  float* st_drop;              // [BH*N] smallest d~ pushed out of a candidate list
+  int4* st_cand;               // [BH*N] up to four candidates (global centroid index, -1 = none)
+  float4* st_dist;             // [BH*N] their d~
   float a_coef, b_coef, s_coef;
 };
 
@@ -191,7 +201,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
   const int64_t left = ntiles_slice - tile0;
   const int ntiles = (int)(left < kTilesPerCta ? left : kTilesPerCta);
   if (ntiles <= 0) return;
-  const int nch = (p.C_pad + kColChunk - 1) / kColChunk;
+  const int nch = (p.cp_pass + kColChunk - 1) / kColChunk;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -214,7 +224,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
     fence_barrier_init();
   }
   for (int c = threadIdx.x; c < kMaxCPad; c += kThreads)
-    cn[c] = c < p.C_pad ? p.cnorm[h * p.C_pad + c] : __int_as_float(0x7f800000);
+    cn[c] = c < p.cp_pass ? p.cnorm[h * p.C_pad + p.c0 + c] : __int_as_float(0x7f800000);
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -229,12 +239,13 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmC);
-      const int nbox = (p.C_pad + p.c_box - 1) / p.c_box;  // whole boxes land, padding included
+      // whole boxes land (rows past the pass see cn = +inf and never win)
+      const int nbox = (p.cp_pass + p.c_box - 1) / p.c_box;
       mbar_arrive_expect_tx(&bars[kBarCFull], nbox * p.c_box * D * 2);
       for (int r = 0; r < nbox * p.c_box; r += p.c_box)
         for (int hf = 0; hf < D / 64; ++hf)
           tma_load_2d(smem + L::kC + hf * L::kCHalf + r * 128, &tmC, &bars[kBarCFull], 64 * hf,
-                      (int32_t)(h * p.C_pad) + r);
+                      (int32_t)(h * p.C_pad + p.c0) + r);
     }
     int issued = 0;
     for (int t = 0; t < ntiles; ++t) {
@@ -273,7 +284,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
             if (!ok) break;
           }
           tc_fence_after();
-          const int n = min(kColChunk, p.C_pad - j * kColChunk);
+          const int n = min(kColChunk, p.cp_pass - j * kColChunk);
           const uint32_t idesc = idesc_f16(128, (uint32_t)n);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -343,7 +354,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         ok = mbar_wait_warp(&bars[kBarTmFull + b], (i >> 1) & 1, abort);
         if (!ok) break;
         tc_fence_after();
-        const int n = min(kColChunk, p.C_pad - j * kColChunk);
+        const int n = min(kColChunk, p.cp_pass - j * kColChunk);
         const uint32_t tbuf = tmem + lane_bits + b * kColChunk;
         // This warpgroup's column groups of the chunk: gg = w + 2u, u = 0..3.
         // Pass 1: minimum of each group (two groups per TMEM wait, four
@@ -375,12 +386,12 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
           tmem_ld32(tbuf + 32 * gg, v);
           tmem_ld_wait();
           if (gmin[u] > thr) continue;
-          const int cbase = j * kColChunk + 32 * gg;
+          const int cbase = j * kColChunk + 32 * gg;  // column of this pass
           uint32_t hit = group_hits(v, cn + cbase, thr);
           if ((hit & (hit - 1)) == 0) {
             // one hit (the usual case): it is the group's minimum column, so
             // its d~ is gmin[u] and needs no extraction from v
-            if (hit) insert(cbase + __ffs(hit) - 1, gmin[u]);
+            if (hit) insert(p.c0 + cbase + __ffs(hit) - 1, gmin[u]);
             hit = 0;
           }
           while (hit) {
@@ -389,7 +400,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
             uint32_t vk = 0;  // v[k] with a static index, so v stays in registers
 #pragma unroll
             for (int kk = 0; kk < 32; ++kk) vk = kk == k ? v[kk] : vk;
-            insert(cbase + k, fmaf(-2.f, __uint_as_float(vk), cn[cbase + k]));
+            insert(p.c0 + cbase + k, fmaf(-2.f, __uint_as_float(vk), cn[cbase + k]));
           }
         }
         tc_fence_before();
@@ -403,25 +414,50 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         xdist[4 * xo + 0] = d0; xdist[4 * xo + 1] = d1; xdist[4 * xo + 2] = d2; xdist[4 * xo + 3] = d3;
       }
       named_bar(1, 256);
-      if (w == 0 && ok) {
-        const float best = fminf(run, xrun[xo]);
-        const float lim = best + margin;
-        const float dropped1 = reinterpret_cast<const float*>(xcnt)[xo];
-        int cs[8];
-        float ds[8];
+      if (w == 0 && ok && valid) {
+        // this warpgroup's list, the other warpgroup's, and (after the first
+        // pass) the state earlier passes carried for the row
+        float best = fminf(run, xrun[xo]);
+        float drop = fminf(dropped, reinterpret_cast<const float*>(xcnt)[xo]);
+        int cs[12];
+        float ds[12];
         cs[0] = c0; cs[1] = c1; cs[2] = c2; cs[3] = c3;
         ds[0] = d0; ds[1] = d1; ds[2] = d2; ds[3] = d3;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           cs[4 + u] = xcand[4 * xo + u];
           ds[4 + u] = xdist[4 * xo + u];
+          cs[8 + u] = -1;
+          ds[8 + u] = inf;
+        }
+        if (p.carry_in) {
+          best = fminf(best, p.st_run[g]);
+          drop = fminf(drop, p.st_drop[g]);
+          const int4 cc = p.st_cand[g];
+          const float4 dd = p.st_dist[g];
+          cs[8] = cc.x; cs[9] = cc.y; cs[10] = cc.z; cs[11] = cc.w;
+          ds[8] = dd.x; ds[9] = dd.y; ds[10] = dd.z; ds[11] = dd.w;
+        }
+        const float lim = best + margin;
+        if (p.carry_out) {
+          // the four smallest candidates within the margin go on; the
+          // smallest one pushed out joins the dropped minimum
+          c0 = c1 = c2 = c3 = -1;
+          d0 = d1 = d2 = d3 = dropped = inf;
+#pragma unroll
+          for (int u = 0; u < 12; ++u)
+            if (cs[u] >= 0 && ds[u] <= lim) insert(cs[u], ds[u]);
+          p.st_run[g] = best;
+          p.st_drop[g] = fminf(drop, dropped);
+          p.st_cand[g] = make_int4(c0, c1, c2, c3);
+          p.st_dist[g] = make_float4(d0, d1, d2, d3);
         }
         int keep = 0, kc[4] = {0, 0, 0, 0};
-        // a candidate pushed out of either list that is still within the
+        // a candidate pushed out of any list that is still within the
         // margin of the row's minimum forces the full decision
-        bool full = cbad || !(margin < inf) || fminf(dropped, dropped1) <= lim;
+        bool full = cbad || !(margin < inf) || drop <= lim;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 12; ++u) {
           const bool live = cs[u] >= 0 && ds[u] <= lim;
           if (live) {
             if (keep < 4) {
@@ -434,7 +470,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
           }
         }
         full = full || keep == 0 || keep > 4;
-        if (valid) {
+        if (!p.carry_out) {
           const int old = old_pre;
           uint8_t kind = kKindFull;
           if (!full && keep == 1) {
@@ -781,6 +817,10 @@ struct TcWs {
   float* cnorm;
   float* cmax;  // [BH] floats, then [BH] ints (cbad): cleared together
   int* cbad;
+  float* st_run;  // row state between passes (C_pad > 512 only)
+  float* st_drop;
+  int4* st_cand;
+  float4* st_dist;
 };
 
 int c_pad_of(int32_t c) { return (int)ceil_div(c, 16) * 16; }
@@ -799,6 +839,11 @@ TcWs carve(Carver& cv, int64_t bh, int64_t n, int32_t d, int32_t c) {
   w.cnorm = cv.take<float>((size_t)bh * cp);
   w.cmax = cv.take<float>((size_t)bh * 2);
   w.cbad = reinterpret_cast<int*>(w.cmax + bh);
+  const bool passes = cp > kMaxCPad;
+  w.st_cand = passes ? cv.take<int4>((size_t)bh * n) : nullptr;
+  w.st_dist = passes ? cv.take<float4>((size_t)bh * n) : nullptr;
+  w.st_run = passes ? cv.take<float>((size_t)bh * n) : nullptr;
+  w.st_drop = passes ? cv.take<float>((size_t)bh * n) : nullptr;
   return w;
 }
 
@@ -844,6 +889,11 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   p.C = c;
   p.C_pad = cp;
   p.c_box = c_box;
+  p.st_run = w.st_run;
+  p.st_drop = w.st_drop;
+  p.st_cand = w.st_cand;
+  p.st_dist = w.st_dist;
+  const int npass = (int)ceil_div(cp, kMaxCPad);
   const double a = 2.0 * (std::ldexp(1.0, -11) + (D + 1) * std::ldexp(1.0, -23)) *
                    (1.0 + std::ldexp(1.0, -11)) * (1.0 + std::ldexp(1.0, -20));
   p.a_coef = (float)(a * (1.0 + 1e-6));
@@ -856,8 +906,14 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   const int64_t crow = bh * (int64_t)c;
   for (int t = 0; t < iters; ++t) {
     p.first = t == 0 ? 1 : 0;
-    km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
-    EAR_TRY(after_launch());
+    for (int pass = 0; pass < npass; ++pass) {  // 512 centroids per pass
+      p.c0 = pass * kMaxCPad;
+      p.cp_pass = std::min(kMaxCPad, cp - p.c0);
+      p.carry_in = pass > 0 ? 1 : 0;
+      p.carry_out = pass + 1 < npass ? 1 : 0;
+      km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
+      EAR_TRY(after_launch());
+    }
     km_resolve<uint16_t, D><<<rgrid, 256, 0, s>>>(X, cent, n, c, rows, labels, p.first, w.kind,
                                                   w.cand, w.from, w.sums, w.cnt);
     EAR_TRY(after_launch());
@@ -873,7 +929,7 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
 }  // namespace
 
 bool kmeans_tc_supported(ear_dtype dt, int32_t d, int32_t c) {
-  return dt == EAR_BF16 && (d == 64 || d == 128) && c_pad_of(c) <= kMaxCPad;
+  return dt == EAR_BF16 && (d == 64 || d == 128) && c_pad_of(c) <= kMaxCTotal;
 }
 
 size_t kmeans_tc_workspace(int64_t bh, int64_t n, int32_t d, int32_t c) {

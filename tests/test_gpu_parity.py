@@ -94,10 +94,14 @@ def test_kmeans_all_iterations(layers, cfg):
 
 
 @pytest.mark.parametrize("n,c,d,iters", [(3001, 500, 64, 4), (2000, 300, 128, 3),
-                                         (777, 17, 128, 5), (4096, 512, 128, 2)])
+                                         (777, 17, 128, 5), (4096, 512, 128, 2),
+                                         (5000, 700, 128, 2), (6000, 1000, 128, 2),
+                                         (3000, 1500, 64, 2), (4096, 2048, 128, 1)])
 def test_kmeans_tensor_core_path_shapes(n, c, d, iters):
-    """bf16 k-means with C <= 512 runs on the tensor cores: two 256-column
-    chunks, a partial last column group, ragged row tiles."""
+    """bf16 k-means with C <= 2048 runs on the tensor cores: two 256-column
+    chunks, a partial last column group, ragged row tiles, and beyond 512
+    centroids passes of 512 with the row state carried between them (the
+    pages' K_C = 1000 among them)."""
     w = gen.MID.with_(heads=2, n=n, d=d, n_centres=max(c // 3, 4), c_q=c, c_k=c, iters=iters)
     L = gen.make_layer(w)
     for it in (1, iters):
