@@ -13,8 +13,10 @@
 //  * pm_gather:    X_perm[r] = X[perm[r]], 16-byte vector copies; a warp
 //                  moves several rows at once (lanes split per row) with four
 //                  row groups in flight per thread.
-//  * pm_segmean:   per-cluster fp32 mean of the permuted rows (v̄, §4.3), a
-//                  fixed-order reduction.
+//  * pm_gather_mean: when the per-cluster means are asked for (v̄, §4.3): one
+//                  block per cluster gathers the cluster's rows into place and
+//                  sums them in a fixed order (per thread over its rows, then
+//                  across the block's row groups), X read once.
 #include "ear_internal.cuh"
 
 namespace ear {
@@ -160,50 +162,93 @@ __global__ void pm_gather(const uint4* __restrict__ X, uint4* __restrict__ Xp,
   }
 }
 
-// block: 256 threads = (256 / (D/4)) row groups x (D/4) column quads
+// one 16-byte piece of a row: its values as floats
+__device__ __forceinline__ void unpack16(const uint4 w, float (&f)[8], const uint16_t*) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f[2 * k] = __uint_as_float(u[k] << 16);
+    f[2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void unpack16(const uint4 w, float (&f)[8], const float*) {
+  f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+  f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+#pragma unroll
+  for (int k = 4; k < 8; ++k) f[k] = 0.f;
+}
+
+// X_perm rows of cluster c = X[perm[r]] for r in [offsets[c], offsets[c+1]),
+// and their fp32 mean in a fixed order.  The offsets must partition [0, N)
+// (offsets[0] = 0, offsets[C] = N, non-decreasing), as ear_permute writes
+// them; a table that does not is latched as an error.  A thread moves one
+// 16-byte piece of a row (kPer values) for every kGroups-th row of the
+// cluster, two rows in flight.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-pm_segmean(const T* __restrict__ Xp, const int32_t* __restrict__ offsets, int64_t N, int C,
-           float* __restrict__ mean, int* status) {
-  constexpr int kQuads = D / 4;
-  constexpr int kGroups = 256 / kQuads;
-  __shared__ float4 part[kGroups][kQuads];
+pm_gather_mean(const T* __restrict__ X, T* __restrict__ Xp, const int32_t* __restrict__ perm,
+               const int32_t* __restrict__ offsets, int64_t N, int C, float* __restrict__ mean,
+               int* status) {
+  constexpr int kPer = 16 / (int)sizeof(T);  // values per 16-byte piece
+  constexpr int kPieces = D / kPer;          // pieces per row
+  constexpr int kGroups = 256 / kPieces;     // rows in flight per block step
+  __shared__ float part[kGroups][D];
   const int64_t h = blockIdx.y;
   const int c = blockIdx.x;
-  const int q = threadIdx.x % kQuads, g = threadIdx.x / kQuads;
+  const int q = threadIdx.x % kPieces, g = threadIdx.x / kPieces;
   const int32_t* oh = offsets + h * (int64_t)(C + 1);
   int32_t r0 = oh[c], r1 = oh[c + 1];
-  if (r0 < 0 || r1 < r0 || r1 > N) {  // offsets passed in by the caller: checked
+  const bool ends_ok = (c > 0 || r0 == 0) && (c < C - 1 || r1 == N);
+  if (r0 < 0 || r1 < r0 || r1 > N || !ends_ok) {
     if (threadIdx.x == 0) latch(status, EAR_ERR_DEVICE);
-    r0 = r1 = 0;
+    if (r0 < 0 || r1 < r0 || r1 > N) r0 = r1 = 0;
   }
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const T* xh = Xp + h * N * D;
-  for (int64_t r = r0 + g; r < r1; r += kGroups) {
-    const T* row = xh + r * D + q * 4;
-    acc.x += Elem<T>::load(row, 0);
-    acc.y += Elem<T>::load(row, 1);
-    acc.z += Elem<T>::load(row, 2);
-    acc.w += Elem<T>::load(row, 3);
+  float acc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  const uint4* xh = reinterpret_cast<const uint4*>(X + h * N * D);
+  uint4* ph = reinterpret_cast<uint4*>(Xp + h * N * D);
+  const int32_t* pp = perm + h * N;
+  for (int64_t r = r0 + g; r < r1; r += 2 * kGroups) {
+    const int64_t ra = r, rb = r + kGroups;
+    const int32_t sa = pp[ra];
+    const int32_t sb = rb < r1 ? pp[rb] : 0;
+    const bool oka = sa >= 0 && sa < N, okb = rb < r1 && sb >= 0 && sb < N;
+    if ((!oka || (rb < r1 && !okb)) && q == 0) latch(status, EAR_ERR_DEVICE);
+    uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = wa;
+    if (oka) wa = xh[(int64_t)sa * kPieces + q];
+    if (okb) wb = xh[(int64_t)sb * kPieces + q];
+    float f[8];
+    if (oka) {
+      ph[ra * kPieces + q] = wa;
+      unpack16(wa, f, X);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += f[k];
+    }
+    if (okb) {
+      ph[rb * kPieces + q] = wb;
+      unpack16(wb, f, X);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += f[k];
+    }
   }
-  part[g][q] = acc;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) part[g][q * kPer + k] = acc[k];
   __syncthreads();
-  if (g == 0) {
-    float4 s = part[0][q];
-    for (int k = 1; k < kGroups; ++k) {
-      s.x += part[k][q].x;
-      s.y += part[k][q].y;
-      s.z += part[k][q].z;
-      s.w += part[k][q].w;
-    }
+  for (int e = threadIdx.x; e < D; e += 256) {
+    float s = part[0][e];
+    for (int k = 1; k < kGroups; ++k) s += part[k][e];
     const int32_t n = r1 - r0;
-    float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (n > 0) {
-      const float fn = (float)n;
-      m = make_float4(s.x / fn, s.y / fn, s.z / fn, s.w / fn);
-    }
-    reinterpret_cast<float4*>(mean + (h * C + c) * (int64_t)D)[q] = m;
+    mean[(h * C + c) * (int64_t)D + e] = n > 0 ? s / (float)n : 0.f;
   }
+}
+
+template <typename T, int D>
+ear_status gather_mean_t(const void* X, void* Xp, const int32_t* perm, const int32_t* offsets,
+                         int64_t bh, int64_t n, int32_t c, float* mean, cudaStream_t s) {
+  pm_gather_mean<T, D><<<dim3((unsigned)c, (unsigned)bh), 256, 0, s>>>(
+      (const T*)X, (T*)Xp, perm, offsets, n, c, mean, device_status_word());
+  return after_launch();
 }
 
 struct PmWs {
@@ -217,14 +262,6 @@ PmWs carve(Carver& cv, int64_t bh, int64_t n, int32_t c) {
   w.hist = cv.take<int32_t>((size_t)bh * c * ntiles);
   w.totals = cv.take<int32_t>((size_t)bh * c);
   return w;
-}
-
-template <typename T, int D>
-ear_status segmean_t(const void* Xp, const int32_t* offsets, int64_t bh, int64_t n, int32_t c,
-                     float* mean, cudaStream_t s) {
-  pm_segmean<T, D><<<dim3((unsigned)c, (unsigned)bh), 256, 0, s>>>((const T*)Xp, offsets, n, c,
-                                                                   mean, device_status_word());
-  return after_launch();
 }
 
 }  // namespace
@@ -259,19 +296,20 @@ ear_status permute_apply_run(const int32_t* perm, const int32_t* offsets, int64_
                              int32_t c, const void* X, void* X_perm, ear_dtype dt, int32_t d,
                              float* seg_mean, cudaStream_t s) {
   int* status = device_status_word();
+  if (seg_mean != nullptr) {  // gather and means in one pass over X
+    if (dt == EAR_F32)
+      return d == 64 ? gather_mean_t<float, 64>(X, X_perm, perm, offsets, bh, n, c, seg_mean, s)
+                     : gather_mean_t<float, 128>(X, X_perm, perm, offsets, bh, n, c, seg_mean, s);
+    return d == 64 ? gather_mean_t<uint16_t, 64>(X, X_perm, perm, offsets, bh, n, c, seg_mean, s)
+                   : gather_mean_t<uint16_t, 128>(X, X_perm, perm, offsets, bh, n, c, seg_mean, s);
+  }
   const int elem = dt == EAR_F32 ? 4 : 2;
   const int row_vecs = d * elem / 16;
   const int64_t rows_total = bh * n;
   const unsigned ggrid = (unsigned)std::min<int64_t>(ceil_div(rows_total, 8), 148 * 64);
   pm_gather<<<ggrid, 256, 0, s>>>((const uint4*)X, (uint4*)X_perm, perm, n, row_vecs, rows_total,
                                   status);
-  EAR_TRY(after_launch());
-  if (seg_mean == nullptr) return EAR_OK;
-  if (dt == EAR_F32)
-    return d == 64 ? segmean_t<float, 64>(X_perm, offsets, bh, n, c, seg_mean, s)
-                   : segmean_t<float, 128>(X_perm, offsets, bh, n, c, seg_mean, s);
-  return d == 64 ? segmean_t<uint16_t, 64>(X_perm, offsets, bh, n, c, seg_mean, s)
-                 : segmean_t<uint16_t, 128>(X_perm, offsets, bh, n, c, seg_mean, s);
+  return after_launch();
 }
 
 }  // namespace ear

@@ -147,7 +147,10 @@ EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int
  *                                   (rows offsets[c] .. offsets[c+1]-1 of
  *                                   X_perm); zero rows for empty clusters
  * Takes no workspace.  A perm entry outside [0, N) latches EAR_ERR_DEVICE and
- * that row is not written.
+ * that row is not written.  With seg_mean, rows are gathered cluster by
+ * cluster, so the offsets must partition [0, N) (offsets[0] = 0,
+ * offsets[C] = N, non-decreasing, as ear_permute writes them); a table that
+ * does not latches EAR_ERR_DEVICE.
  */
 EAR_API ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_t bh,
                                      int64_t n, int32_t c, const void* X, void* X_perm,
