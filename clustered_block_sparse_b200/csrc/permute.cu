@@ -48,13 +48,19 @@ pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int nti
   int32_t* hh = hist + h * (int64_t)C * ntiles;  // [tile][cluster]
   int32_t* th = totals + h * (int64_t)C;
   // per cluster: exclusive prefix over tiles, total in `totals` (consecutive
-  // threads read consecutive clusters of one tile)
+  // threads read consecutive clusters of one tile; 16 tiles' counts are
+  // loaded before they are summed)
   for (int c = tid; c < C; c += 1024) {
     int32_t run = 0;
-    for (int t = 0; t < ntiles; ++t) {
-      const int32_t v = hh[(int64_t)t * C + c];
-      hh[(int64_t)t * C + c] = run;
-      run += v;
+    for (int t0 = 0; t0 < ntiles; t0 += 16) {
+      int32_t v[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = t0 + k < ntiles ? hh[(int64_t)(t0 + k) * C + c] : 0;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (t0 + k < ntiles) hh[(int64_t)(t0 + k) * C + c] = run;
+        run += v[k];
+      }
     }
     th[c] = run;
   }
@@ -90,17 +96,14 @@ pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int nti
     __syncthreads();
   }
   if (tid == 0) oh[C] = carry;
-  __syncthreads();
-  // cursor of every (cluster, tile) = cluster offset + earlier tiles' members
-  for (int c = tid; c < C; c += 1024) {
-    const int32_t o = oh[c];
-    for (int t = 0; t < ntiles; ++t) hh[(int64_t)t * C + c] += o;
-  }
+  // the cursor of (cluster, tile) is offsets[cluster] + hist[tile][cluster]:
+  // pm_scatter adds the offset
 }
 
 __global__ void __launch_bounds__(kTile)
 pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
-           int32_t* __restrict__ cursor, int32_t* __restrict__ perm) {
+           int32_t* __restrict__ cursor, const int32_t* __restrict__ offsets,
+           int32_t* __restrict__ perm) {
   const int64_t h = blockIdx.y;
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -114,13 +117,14 @@ pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
   const int leader = __ffs(group) - 1;
   const int before = __popc(group & ((1u << lane) - 1u));
   int32_t* cur = cursor + (h * ntiles + tile) * (int64_t)C + (c < 0 ? 0 : c);
+  const int32_t off = c >= 0 ? offsets[h * (int64_t)(C + 1) + c] : 0;
   for (int w = 0; w < 32; ++w) {
     if (wid == w) {
       int32_t base = 0;
       if (lane == leader && c >= 0) base = *cur;
       base = __shfl_sync(0xffffffffu, base, leader);
       if (c >= 0) {
-        perm[h * N + base + before] = (int32_t)i;
+        perm[h * N + off + base + before] = (int32_t)i;
         if (lane == leader) *cur = base + __popc(group);
       }
     }
@@ -286,7 +290,7 @@ ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, 
   EAR_TRY(after_launch());
   pm_scan<<<(unsigned)bh, 1024, 0, s>>>(w.hist, w.totals, c, ntiles, offsets);
   EAR_TRY(after_launch());
-  pm_scatter<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, perm);
+  pm_scatter<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, offsets, perm);
   EAR_TRY(after_launch());
   if (X == nullptr) return EAR_OK;
   return permute_apply_run(perm, offsets, bh, n, c, X, X_perm, dt, d, seg_mean, s);
