@@ -100,13 +100,24 @@ pm_scan(int32_t* __restrict__ hist, int32_t* __restrict__ totals, int C, int nti
   // pm_scatter adds the offset
 }
 
+// Stable scatter of one tile: the tile's 32 warps take turns; a warp's rows
+// of one cluster go to consecutive places after those of earlier warps and
+// tiles.  SHARED: the tile's cursors (offset + earlier tiles' members) live in
+// shared memory, else in the global cursor table.
+template <bool SHARED>
 __global__ void __launch_bounds__(kTile)
 pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
            int32_t* __restrict__ cursor, const int32_t* __restrict__ offsets,
            int32_t* __restrict__ perm) {
+  extern __shared__ int32_t scur[];
   const int64_t h = blockIdx.y;
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (SHARED) {
+    for (int k = tid; k < C; k += kTile)
+      scur[k] = offsets[h * (int64_t)(C + 1) + k] + cursor[(h * ntiles + tile) * (int64_t)C + k];
+    __syncthreads();
+  }
   const int64_t i = (int64_t)tile * kTile + tid;
   int c = -1;
   if (i < N) {
@@ -116,8 +127,9 @@ pm_scatter(const int32_t* __restrict__ labels, int64_t N, int C, int ntiles,
   const unsigned group = __match_any_sync(0xffffffffu, c);
   const int leader = __ffs(group) - 1;
   const int before = __popc(group & ((1u << lane) - 1u));
-  int32_t* cur = cursor + (h * ntiles + tile) * (int64_t)C + (c < 0 ? 0 : c);
-  const int32_t off = c >= 0 ? offsets[h * (int64_t)(C + 1) + c] : 0;
+  int32_t* cur = SHARED ? scur + (c < 0 ? 0 : c)
+                        : cursor + (h * ntiles + tile) * (int64_t)C + (c < 0 ? 0 : c);
+  const int32_t off = (!SHARED && c >= 0) ? offsets[h * (int64_t)(C + 1) + c] : 0;
   for (int w = 0; w < 32; ++w) {
     if (wid == w) {
       int32_t base = 0;
@@ -290,7 +302,11 @@ ear_status permute_run(const int32_t* labels, int64_t bh, int64_t n, int32_t c, 
   EAR_TRY(after_launch());
   pm_scan<<<(unsigned)bh, 1024, 0, s>>>(w.hist, w.totals, c, ntiles, offsets);
   EAR_TRY(after_launch());
-  pm_scatter<<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, offsets, perm);
+  const size_t scur_bytes = sizeof(int32_t) * (size_t)c;
+  if (scur_bytes <= 48 * 1024)
+    pm_scatter<true><<<tgrid, kTile, scur_bytes, s>>>(labels, n, c, ntiles, w.hist, offsets, perm);
+  else
+    pm_scatter<false><<<tgrid, kTile, 0, s>>>(labels, n, c, ntiles, w.hist, offsets, perm);
   EAR_TRY(after_launch());
   if (X == nullptr) return EAR_OK;
   return permute_apply_run(perm, offsets, bh, n, c, X, X_perm, dt, d, seg_mean, s);
