@@ -12,7 +12,8 @@
 // digit at which the running cost crosses the remaining budget.  Ratios are
 // correctly rounded fp64 divisions, so the order matches a host fp64 sort.
 //
-// Main path (C_q <= 1024 and C_q C_k <= 8 x kKeysPerCta): one cluster of 8 CTAs per slice.
+// Main path (C_q <= 512 and C_q C_k <= 8 x kKeysPerCta): one cluster of 8 CTAs of 512 threads
+// per slice.
 // Each CTA keeps the keys of its eighth of the blocks in shared memory; in
 // each pass every CTA adds its costs into the histogram of CTA 0 through
 // distributed shared memory (a warp whose lanes share one digit adds them in
@@ -254,6 +255,7 @@ rt_route(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
 
 constexpr int kCluster = 8;
 constexpr int kKeysPerCta = 16384;  // 128 KB of keys per CTA
+constexpr int kCThreads = 512;      // threads of a cluster CTA: two CTAs fit one SM
 
 namespace cg = cooperative_groups;
 
@@ -263,7 +265,7 @@ size_t cluster_smem(int Cq, int Ck, int64_t per) {
   return (size_t)per * 8 + (size_t)(Cq + Ck) * 4 + (size_t)(Cq + 1) * 8;
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
 rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all,
                  const int32_t* __restrict__ kn_all, int Cq, int Ck, int64_t budget, int mode,
                  uint8_t* __restrict__ exact_all, int32_t* __restrict__ blk_off_all,
@@ -295,9 +297,9 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
   int32_t* blk_off = blk_off_all + h * (int64_t)(Cq + 1);
   int32_t* blk_list = blk_list_all + h * (int64_t)nblk;
 
-  for (int i = tid; i < Cq; i += kThreads) sqn[i] = qn_all[h * Cq + i];
-  for (int i = tid; i < Ck; i += kThreads) skn[i] = kn_all[h * Ck + i];
-  for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+  for (int i = tid; i < Cq; i += kCThreads) sqn[i] = qn_all[h * Cq + i];
+  for (int i = tid; i < Ck; i += kCThreads) skn[i] = kn_all[h * Ck + i];
+  for (int i = tid; i < 256; i += kCThreads) hist[i] = 0;
   if (tid == 0) {
     s_phi = 0;
     s_plo = 0;
@@ -306,7 +308,7 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
     s_total = 0;
   }
   __syncthreads();
-  for (int idx = i0 + tid; idx < i1; idx += kThreads) {
+  for (int idx = i0 + tid; idx < i1; idx += kCThreads) {
     Key k;
     unsigned long long c = 0;
     skey[idx - i0] = block_key(Eh, sqn, skn, Ck, mode, idx, k, c) ? k.hi : 0ull;
@@ -319,7 +321,7 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
   for (int pass = 0; pass < 12; ++pass) {
     const uint64_t phi = *phi0;
     const uint32_t plo = *plo0;
-    for (int base = i0; base < i1; base += kThreads) {
+    for (int base = i0; base < i1; base += kCThreads) {
       const int idx = base + tid;
       Key k;
       unsigned long long c = 0;
@@ -391,7 +393,7 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
   const uint64_t kstar_hi = *phi0;
   const uint32_t kstar_lo = *plo0;
   // mark this CTA's blocks
-  for (int idx = i0 + tid; idx < i1; idx += kThreads) {
+  for (int idx = i0 + tid; idx < i1; idx += kCThreads) {
     const int a = idx / Ck, b = idx - a * Ck;
     const bool live = (int64_t)sqn[a] * (int64_t)skn[b] > 0;
     Key k;
@@ -403,7 +405,7 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
     pairs[h] = all_fit ? (int64_t)s_total : (int64_t)(budget - s_rem);
   cl.sync();  // every CTA's marks are visible to the cluster
   // exact key clusters per query cluster, and their offsets (every CTA)
-  for (int a = wid; a < Cq; a += kThreads / 32) {
+  for (int a = wid; a < Cq; a += kCThreads / 32) {
     int cnt = 0;
     for (int b = lane; b < Ck; b += 32) cnt += exact[(int64_t)a * Ck + b];
 #pragma unroll
@@ -411,7 +413,7 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
     if (lane == 0) scnt[a] = cnt;
   }
   __syncthreads();
-  {  // exclusive scan of the counts (the cluster path has C_q <= kThreads)
+  {  // exclusive scan of the counts (the cluster path has C_q <= kCThreads)
     const int a = tid;
     const int32_t v = a < Cq ? scnt[a] : 0;
     int32_t x = v;
@@ -438,9 +440,9 @@ rt_route_cluster(const float* __restrict__ E, const int32_t* __restrict__ qn_all
     __syncthreads();
   }
   if (rank == 0)
-    for (int a = tid; a <= Cq; a += kThreads) blk_off[a] = soff[a];
+    for (int a = tid; a <= Cq; a += kCThreads) blk_off[a] = soff[a];
   // lists of this CTA's share of the query clusters (a = rank, rank + 8, ...)
-  for (int a = rank + kCluster * wid; a < Cq; a += kCluster * (kThreads / 32)) {
+  for (int a = rank + kCluster * wid; a < Cq; a += kCluster * (kCThreads / 32)) {
     int32_t pos = soff[a];
     for (int b0 = 0; b0 < Ck; b0 += 32) {
       const int b = b0 + lane;
@@ -461,7 +463,7 @@ constexpr size_t kClusterSmemMax = 200 * 1024;
 bool use_cluster(int32_t c_q, int32_t c_k) {
   const int64_t nblk = (int64_t)c_q * c_k;
   const int64_t per = (nblk + kCluster - 1) / kCluster;
-  return c_q <= kThreads && per <= kKeysPerCta && cluster_smem(c_q, c_k, per) <= kClusterSmemMax;
+  return c_q <= kCThreads && per <= kKeysPerCta && cluster_smem(c_q, c_k, per) <= kClusterSmemMax;
 }
 }  // namespace
 
@@ -480,7 +482,7 @@ ear_status route_run(const float* E, const int32_t* qn, const int32_t* kn, int64
     const size_t smem = cluster_smem(c_q, c_k, per);
     EAR_CUDA(cudaFuncSetAttribute(rt_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem));
-    rt_route_cluster<<<dim3(kCluster, (unsigned)bh), kThreads, smem, s>>>(
+    rt_route_cluster<<<dim3(kCluster, (unsigned)bh), kCThreads, smem, s>>>(
         E, qn, kn, c_q, c_k, budget, mode, exact, blk_off, blk_list, pairs);
     return after_launch();
   }
