@@ -128,19 +128,22 @@ def attention_bytes(w) -> float:
     return 4.0 * w.heads * w.n * w.d * (2 if w.dtype == "bf16" else 4)
 
 
-def stage_bytes(w) -> dict:
+def stage_bytes(w, layout="permuted") -> dict:
     """Algorithmic HBM bytes of each stage (what it must move at least once):
     k-means reads Q and K once per iteration (labels are 4 bytes a row);
-    permute reads and writes Q, K and V (plus labels in, permutation out);
-    the probe reads the permuted keys once and writes E; the route reads E
-    and writes the mask and lists; attention reads Q, K, V and writes O."""
+    permute reads and writes Q, K and V (plus labels in, permutation out) --
+    gathered, it reads only V (for v̄) besides the labels and permutations;
+    the probe reads the keys once and writes E; the route reads E and writes
+    the mask and lists; attention reads Q, K, V and writes O."""
     el = 2 if w.dtype == "bf16" else 4
     tok = w.heads * w.n * w.d * el
     rows = w.heads * w.n
     blocks = w.heads * w.c_q * w.c_k
+    permute = (3.0 * 2 * tok + 2 * 3 * 4 * rows if layout == "permuted"
+               else tok + 2 * 2 * 4 * rows + 4 * rows)
     return {
         "kmeans": 2.0 * w.iters * (tok + 4 * rows),
-        "permute": 3.0 * 2 * tok + 2 * 3 * 4 * rows,
+        "permute": permute,
         "probe": tok + 4.0 * blocks,
         "route": 4.0 * blocks + 1.0 * blocks + 4.0 * blocks,
         "attention": attention_bytes(w),
@@ -201,7 +204,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/layer",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": value,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, args.gpus),
+        "data": "synthetic", "config": config_of(w, args.gpus, args.layout),
         "cpu_baseline": {"value": value, "unit": "ms/layer", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "ms/layer", "h2d_bytes_per_step": 0,
@@ -230,10 +233,13 @@ def recorded_traffic(heads: int):
     return per_head * heads if sha == cur else None
 
 
-def config_of(w, n_gpus):
+def config_of(w, n_gpus, layout="permuted"):
     return {"workload": w.name, "heads": w.heads, "n_q": w.n, "n_k": w.n, "d": w.d,
             "c_q": w.c_q, "c_k": w.c_k, "kmeans_iters": w.iters, "density": w.density,
             "ratio_mode": 0, "compensate": True,
+            "layout": ("gathered: Q, K, V stay in token order; probe and attention read rows "
+                       "through the permutations (TMA tile::gather4)" if layout == "gathered"
+                       else "permuted: cluster-contiguous copies of Q, K, V"),
             "l2": "inputs larger than L2 (Q, K, V per step >> 126 MB); no flush",
             "parallelism": f"{n_gpus} independent replica(s), one layer per rank, no collective"}
 
@@ -273,6 +279,7 @@ def run_ear(args, w):
     ki = torch.from_numpy(layer.k_init).to(dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
+    gathered = args.layout == "gathered"
 
     def step(ev=None):
         """One layer; `ev` = 6 events recorded at the stage boundaries."""
@@ -281,15 +288,24 @@ def run_ear(args, w):
         qc, ql, qn = ear.ear_kmeans(q, qi, w.iters)
         kc, kl, kn = ear.ear_kmeans(k, ki, w.iters)
         rec(1)
-        qp, qo, qx, _ = ear.ear_permute(ql, w.c_q, q)
-        kp, ko, kx, _ = ear.ear_permute(kl, w.c_k, k)
-        vx, vm = ear.ear_permute_apply(kp, ko, v, seg_mean=True)
+        if gathered:
+            qp, qo, _, _ = ear.ear_permute(ql, w.c_q)
+            kp, ko, _, _ = ear.ear_permute(kl, w.c_k)
+            _, vm = ear.ear_permute_apply(kp, ko, v, seg_mean=True, write_perm=False)
+        else:
+            qp, qo, qx, _ = ear.ear_permute(ql, w.c_q, q)
+            kp, ko, kx, _ = ear.ear_permute(kl, w.c_k, k)
+            vx, vm = ear.ear_permute_apply(kp, ko, v, seg_mean=True)
         rec(2)
-        e = ear.ear_probe(qc, qn, kc, kx, ko)
+        e = (ear.ear_probe_gather(qc, qn, kc, k, kp, ko) if gathered
+             else ear.ear_probe(qc, qn, kc, kx, ko))
         rec(3)
         exact, bo, bl, pairs = ear.ear_route(e, qn, kn, w.n, w.n, w.density)
         rec(4)
-        ear.ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, out=out)
+        if gathered:
+            ear.ear_attention_gather(q, k, v, qo, ko, qp, kp, kc, vm, exact, bo, bl, out=out)
+        else:
+            ear.ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, out=out)
         rec(5)
         return exact, qo, kn, pairs
 
@@ -342,7 +358,7 @@ def run_ear(args, w):
     # the attention kernel runs at full clock inside the step (see "clocks"), so
     # the burst figure is its denominator; the sustained one is reported beside it
     peak = peaks["bf16_tflops"]
-    sb = stage_bytes(w)
+    sb = stage_bytes(w, args.layout)
     hbm = {st: {"algorithmic_gb": sb[st] / 1e9,
                 "achieved_gbs": sb[st] / (stage_ms[st] * 1e-3) / 1e9,
                 "frac_of_measured_hbm": sb[st] / (stage_ms[st] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
@@ -367,7 +383,7 @@ def run_ear(args, w):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded Gaussian-mixture / smoothed-field tokens; no model weights)",
-        "config": config_of(w, world),
+        "config": config_of(w, world, args.layout),
         "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
         "overhead_frac": (stage_ms["kmeans"] + stage_ms["probe"] + stage_ms["route"]) /
                          sum(stage_ms.values()),
@@ -439,7 +455,8 @@ def time_e2e(args, w, layer, ear, dev, tdt, stream):
         stream.wait_event(uploaded[sl])
         with torch.cuda.stream(stream):
             res = ear.ear_layer(bufs[sl]["q"], bufs[sl]["k"], bufs[sl]["v"], ibufs[sl]["q_init"],
-                                ibufs[sl]["k_init"], w.iters, w.density)
+                                ibufs[sl]["k_init"], w.iters, w.density,
+                                gather=args.layout == "gathered")
         consumed[sl].record(stream)
         down.wait_event(consumed[sl])
         with torch.cuda.stream(down):
@@ -727,6 +744,8 @@ def main(argv=None):
                     help="run a quality study instead of the timing line")
     ap.add_argument("--c-q", type=int, default=None, help="query clusters of a study")
     ap.add_argument("--c-k", type=int, default=None, help="key clusters of a study")
+    ap.add_argument("--layout", choices=("permuted", "gathered"), default="permuted",
+                    help="permuted copies of Q, K, V, or reads through the permutations")
     args = ap.parse_args(argv)
     if args.study == "skew":
         return run_skew_study(args)

@@ -19,7 +19,8 @@ EAR_COMPENSATE = 1
 EAR_PROBE_LOGIT, EAR_PROBE_WEIGHTS, EAR_PROBE_VALUE = 0, 1, 2
 
 EXPORTED = ("ear_status_string", "ear_workspace_bytes", "ear_kmeans", "ear_permute",
-            "ear_permute_apply", "ear_permute_static", "ear_probe", "ear_route", "ear_attention",
+            "ear_permute_apply", "ear_permute_static", "ear_probe", "ear_probe_gather", "ear_route",
+            "ear_attention", "ear_attention_gather",
             "ear_route_rows", "ear_topp_budget", "ear_uniform_budget", "ear_cluster_stats",
             "ear_normalizer_change",
             "ear_get_device_status", "ear_launch_count")
@@ -60,6 +61,9 @@ def lib() -> ctypes.CDLL:
                                      _i32, _vp, _vp]
     L.ear_probe.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _vp, _i64, _i64, _i32, _i32, _i32,
                             ctypes.c_float, _i32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.ear_probe_gather.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_int, _vp, _i64, _i64, _i32,
+                                   _i32, _i32, ctypes.c_float, _i32, _vp, _vp, _vp, _vp,
+                                   ctypes.c_size_t, _vp]
     L.ear_route.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, ctypes.c_double, _i32,
                             _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     L.ear_route_rows.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -73,14 +77,17 @@ def lib() -> ctypes.CDLL:
     L.ear_attention.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, _i64, _i64, _i64, _i32, _i32, _i32, ctypes.c_float, _i32,
                                 _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.ear_attention_gather.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
+                                       ctypes.c_float, _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     L.ear_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), _vp]
     L.ear_launch_count.argtypes = []
     L.ear_launch_count.restype = ctypes.c_uint64
     for name in ("ear_workspace_bytes", "ear_kmeans", "ear_permute", "ear_permute_apply",
                  "ear_permute_static",
-                 "ear_probe", "ear_route", "ear_route_rows", "ear_topp_budget",
+                 "ear_probe", "ear_probe_gather", "ear_route", "ear_route_rows", "ear_topp_budget",
                  "ear_uniform_budget", "ear_cluster_stats", "ear_normalizer_change",
-                 "ear_attention", "ear_get_device_status"):
+                 "ear_attention", "ear_attention_gather", "ear_get_device_status"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L

@@ -77,7 +77,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 at_simt(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
         const int32_t* __restrict__ q_off_all, const int32_t* __restrict__ k_off_all,
-        const int32_t* __restrict__ q_perm_all, const float* __restrict__ kc_all,
+        const int32_t* __restrict__ q_perm_all, const int32_t* __restrict__ k_perm_all,
+        const float* __restrict__ kc_all,
         const float* __restrict__ vc_all, const uint8_t* __restrict__ exact_all,
         const int32_t* __restrict__ blk_off_all, const int32_t* __restrict__ blk_list_all,
         const int2* __restrict__ items_all, const int32_t* __restrict__ count_all,
@@ -112,9 +113,23 @@ at_simt(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ 
   const T* Vh = V + h * Nk * D;
   const float qscale = scale * kLog2e;
 
+  // k_perm_all != nullptr (gather): Q, K and V are in original token order;
+  // permuted row r is original row q_perm[r] / k_perm[r].
+  const int32_t* qp = k_perm_all != nullptr ? q_perm_all + h * Nq : nullptr;
+  const int32_t* kp = k_perm_all != nullptr ? k_perm_all + h * Nk : nullptr;
+  auto src_row = [&](const int32_t* perm, int64_t r, int64_t n) -> int64_t {
+    if (perm == nullptr) return r;
+    const int32_t o = perm[r];
+    if (o < 0 || o >= n) {
+      latch(status, EAR_ERR_DEVICE);
+      return -1;
+    }
+    return o;
+  };
   for (int e = tid; e < kTile * D; e += kThreads) {
     const int rr = e / D, k = e % D;
-    qs[rr * QS + k] = rr < nrows ? Elem<T>::load(Qh, (int64_t)(row0 + rr) * D + k) * qscale : 0.f;
+    const int64_t src = rr < nrows ? src_row(qp, row0 + rr, Nq) : -1;
+    qs[rr * QS + k] = src >= 0 ? Elem<T>::load(Qh, src * D + k) * qscale : 0.f;
   }
 
   float m = -INFINITY, l = 0.f;
@@ -186,9 +201,9 @@ at_simt(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ 
       __syncthreads();
       for (int x = tid; x < kKeys * D; x += kThreads) {
         const int j = x / D, k = x % D;
-        const bool ok = j < nv;
-        ks[j * KS + k] = ok ? Elem<T>::load(Kh, (int64_t)(j0 + j) * D + k) : 0.f;
-        vs[j * KS + k] = ok ? Elem<T>::load(Vh, (int64_t)(j0 + j) * D + k) : 0.f;
+        const int64_t src = j < nv ? src_row(kp, j0 + j, Nk) : -1;
+        ks[j * KS + k] = src >= 0 ? Elem<T>::load(Kh, src * D + k) : 0.f;
+        vs[j * KS + k] = src >= 0 ? Elem<T>::load(Vh, src * D + k) : 0.f;
       }
       if (tid < kKeys) bias[tid] = 0.f;
       consume(nv);
@@ -245,7 +260,7 @@ ear_status simt_t(const AttnArgs& a, const int2* items, const int32_t* count, in
                                 (int)smem));
   const dim3 grid((unsigned)max_items, (unsigned)a.bh);
   at_simt<T, D><<<grid, kThreads, smem, s>>>(
-      (const T*)a.Q, (const T*)a.K, (const T*)a.V, a.q_off, a.k_off, a.q_perm, a.k_cent,
+      (const T*)a.Q, (const T*)a.K, (const T*)a.V, a.q_off, a.k_off, a.q_perm, a.k_perm, a.k_cent,
       a.v_cent, a.exact, a.blk_off, a.blk_list, items, count, max_items, a.n_q, a.n_k, a.c_q,
       a.c_k, a.scale, a.flags & EAR_COMPENSATE, (T*)a.O, a.lse, device_status_word());
   return after_launch();

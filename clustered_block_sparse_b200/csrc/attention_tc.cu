@@ -22,7 +22,17 @@
 //   warp 0      TMA producer: Q tiles once, then chunk boxes into a 4-stage
 //               ring.  It publishes each stage's chunk descriptor (box count,
 //               valid rows per box, centroid or not, bias) in shared memory
-//               and ends the sequence with an empty descriptor.
+//               and ends the sequence with an empty descriptor.  With G
+//               (gather) Q, K and V stay in their original token order: the
+//               producer walks the box sequence two chunks ahead of the ring,
+//               keeping each chunk's descriptor in a small shared-memory ring
+//               and fetching the original index of each of its permuted rows
+//               (k_perm) with 4-byte cp.async copies into a matching index
+//               ring, so the index latency overlaps the chunks before it; at
+//               issue the lanes check and convert the indices and the elected
+//               lane fetches rows four at a time with TMA tile::gather4 into
+//               the same swizzled layout (§3.1's permutation folded into the
+//               loads; no permuted copies).
 //   warp 1      MMA issuer (one elected lane of the warp): S_t = Q_t K^T into
 //               one of two TMEM buffers per tile, then O_t += P_t V with P_t
 //               read from TMEM.  Issue order
@@ -53,6 +63,8 @@ constexpr int kBox = 32;                 // rows per TMA box
 constexpr int kBoxes = 2;                // boxes per chunk
 constexpr int kChunk = kBox * kBoxes;    // keys per chunk
 constexpr int kStages = 4;               // K/V ring depth (chunks)
+constexpr int kLook = 2;                 // gather: chunks walked ahead of the issue
+constexpr int kRing = 4;                 // gather: descriptor / index ring (> kLook)
 constexpr int kSBufs = 2;                // S buffers per tile: Q K^T of chunk c+1 runs
                                          // while the softmax works on chunk c
 constexpr int kThreads = 384;
@@ -91,6 +103,11 @@ struct ChunkInfo {
   int32_t valid[kBoxes]; // valid rows of each box (1..32)
 };
 
+// Gather: a chunk walked ahead of its issue (the producer's own ring).
+struct AheadDesc {
+  int32_t nbox, comp, r0, r1, v0, v1, comp_first, pad;
+};
+
 template <int D>
 struct Layout {
   static constexpr int kHalfBytes = kTileRows * 128;  // Q tile: 128 rows x 64 bf16 per half
@@ -105,7 +122,10 @@ struct Layout {
   static constexpr int kList = kInfo + kStages * 32;              // unit's exact key clusters
   static constexpr int kKoff = kList + kTableMax * 4;             // slice's key offsets
   static constexpr int kExact = kKoff + kTableMax * 4;            // unit's row of the mask
-  static constexpr int kBar = kExact + kTableMax;
+  static constexpr int kQIdx = kExact + kTableMax;                // gather: Q row coordinates
+  static constexpr int kGIdx = kQIdx + kUnitRows * 4;             // gather: kRing chunks' K / V rows
+  static constexpr int kAhead = kGIdx + kRing * kChunk * 4;       // gather: kRing AheadDesc
+  static constexpr int kBar = kAhead + kRing * (int)sizeof(AheadDesc);
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -114,6 +134,7 @@ struct TcParams {
   const int32_t* q_off;
   const int32_t* k_off;
   const int32_t* q_perm;
+  const int32_t* k_perm;  // gather: original index of each permuted key
   const uint8_t* exact;
   const int32_t* blk_off;
   const int32_t* blk_list;
@@ -274,11 +295,11 @@ __device__ __forceinline__ unsigned long long box_exp_c(const uint32_t (&v)[32],
   return add2(sum0, sum1);
 }
 
-template <int D>
+template <int D, bool G>
 __device__ __forceinline__ void producer_role(
     const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
     const CUtensorMap& tmKc, const CUtensorMap& tmVc, const TcParams& p, uint8_t* smem, int64_t h,
-    int a, int32_t row0, int ntiles, int lane, volatile int* abort) {
+    int a, int32_t row0, int ntiles, int qrows, int lane, volatile int* abort) {
   using L = Layout<D>;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   float* bias = reinterpret_cast<float*>(smem + L::kBias);
@@ -288,15 +309,32 @@ __device__ __forceinline__ void producer_role(
     const uint8_t* exact_row = p.exact + (h * p.Cq + a) * (int64_t)p.Ck;
     const int32_t* koff = p.k_off + h * (int64_t)(p.Ck + 1);
     const bool leader = elect_one();  // issues the TMA copies (operands stay warp-uniform)
+    int32_t* qidx = reinterpret_cast<int32_t*>(smem + L::kQIdx);
+    if (G) {  // the unit's query rows; rows past the unit repeat its last row
+      for (int r = lane; r < ntiles * kTileRows; r += 32)
+        qidx[r] = gather_row(p.q_perm, h * p.Nq + row0 + min(r, qrows - 1), h, p.Nq, p.status);
+      __syncwarp();
+    }
     if (leader) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bars[kBarQFull], ntiles * L::kTileBytes);
-      for (int t = 0; t < ntiles; ++t)
-        for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_2d(smem + L::kQ + t * L::kTileBytes + hf * L::kHalfBytes, &tmQ,
-                      &bars[kBarQFull], 64 * hf, (int32_t)(h * p.Nq) + row0 + kTileRows * t);
+      for (int t = 0; t < ntiles; ++t) {
+        uint8_t* qdst = smem + L::kQ + t * L::kTileBytes;
+        if (G) {
+          for (int g = 0; g < kTileRows / 4; ++g) {
+            const int4 rr = *reinterpret_cast<const int4*>(qidx + t * kTileRows + 4 * g);
+            for (int hf = 0; hf < D / 64; ++hf)
+              tma_gather4(qdst + hf * L::kHalfBytes + g * 4 * 128, &tmQ, &bars[kBarQFull],
+                          64 * hf, rr);
+          }
+        } else {
+          for (int hf = 0; hf < D / 64; ++hf)
+            tma_load_2d(qdst + hf * L::kHalfBytes, &tmQ, &bars[kBarQFull], 64 * hf,
+                        (int32_t)(h * p.Nq) + row0 + kTileRows * t);
+        }
+      }
     }
     // Stage the unit's block list and the slice's key offsets in shared memory
     // (the box walk below would otherwise chase them through L2 per block).
@@ -345,13 +383,44 @@ __device__ __forceinline__ void producer_role(
         have = it.next(brow, bval, bcomp);
       }
     };
-    gather();
+    // G: chunk j walked ahead -> descriptor ring slot j % kRing, and its rows'
+    // k_perm entries copied asynchronously into the index ring (rows past a
+    // box's valid count repeat its last row); one commit group per chunk
+    AheadDesc* ahead = reinterpret_cast<AheadDesc*>(smem + L::kAhead);
+    int32_t* gring = reinterpret_cast<int32_t*>(smem + L::kGIdx);
+    auto walk_ahead = [&](int j) {
+      gather();
+      const int slot = j % kRing;
+      if (lane == 0) ahead[slot] = AheadDesc{nbox, comp, r0, r1, v0, v1, comp_first, 0};
+      if (!comp) {
+        const int32_t* kp = p.k_perm + h * p.Nk;
+        if (nbox > 0) cp_async4(gring + slot * kChunk + lane, kp + r0 + min(lane, v0 - 1));
+        if (nbox > 1) cp_async4(gring + slot * kChunk + 32 + lane, kp + r1 + min(lane, v1 - 1));
+      }
+      cp_async_commit();
+    };
+    if (G) {
+      for (int j = 0; j < kLook; ++j) walk_ahead(j);
+    } else {
+      gather();
+    }
     int issued = 0;
     for (int c = 0;; ++c) {
       const int s = c % kStages;
       if (c >= kStages && !mbar_wait(&bars[kBarKvEmpty + s], ((c / kStages) - 1) & 1, abort))
         break;
       issued = c + 1;
+      if (G) {  // this chunk's descriptor, walked kLook chunks ago
+        __syncwarp();
+        const AheadDesc d = ahead[c % kRing];
+        nbox = d.nbox;
+        comp = d.comp;
+        r0 = d.r0;
+        r1 = d.r1;
+        v0 = d.v0;
+        v1 = d.v1;
+        comp_first = d.comp_first;
+      }
       if (comp) {  // bias of the chunk's columns (centroids comp_first ...)
         for (int j = lane; j < kChunk; j += 32) {
           float bv = -INFINITY;
@@ -377,7 +446,35 @@ __device__ __forceinline__ void producer_role(
         else
           mbar_arrive_expect_tx(&bars[kBarKvFull + s], 2 * (comp ? 2 : nbox) * kBox * D * 2);
       }
-      {
+      if (G && !comp) {
+        // this lane's index copies of chunk c have landed (kLook - 1 later chunks may not);
+        // each lane checks its two entries and turns them into row coordinates
+        cp_async_wait<kLook - 1>();
+        int32_t* gidx = gring + (c % kRing) * kChunk;
+        for (int k = 0; k < nbox; ++k) {
+          int32_t o = gidx[lane + 32 * k];
+          if (o < 0 || o >= p.Nk) {
+            latch(p.status, EAR_ERR_DEVICE);
+            o = 0;
+          }
+          gidx[lane + 32 * k] = (int32_t)(h * p.Nk) + o;
+        }
+        __syncwarp();
+        uint8_t* kdst = smem + L::kK + s * L::kStageBytes;
+        uint8_t* vdst = smem + L::kV + s * L::kStageBytes;
+        if (leader) {
+          for (int g = 0; g < nbox * (kBox / 4); ++g) {
+            const int4 rr = *reinterpret_cast<const int4*>(gidx + 4 * g);
+#pragma unroll
+            for (int hf = 0; hf < D / 64; ++hf) {
+              tma_gather4(kdst + hf * L::kSHalf + g * 4 * 128, &tmK, &bars[kBarKvFull + s],
+                          64 * hf, rr);
+              tma_gather4(vdst + hf * L::kSHalf + g * 4 * 128, &tmV, &bars[kBarKvFull + s],
+                          64 * hf, rr);
+            }
+          }
+        }
+      } else {
         const CUtensorMap* mk = comp ? &tmKc : &tmK;
         const CUtensorMap* mv = comp ? &tmVc : &tmV;
         const int32_t base = comp ? (int32_t)(h * p.Ck_pad) : (int32_t)(h * p.Nk);
@@ -400,8 +497,12 @@ __device__ __forceinline__ void producer_role(
       }
       __syncwarp();
       if (nbox == 0) break;
-      gather();
+      if (G)
+        walk_ahead(c + kLook);
+      else
+        gather();
     }
+    if (G) cp_async_wait_all();  // no index copy outlives the producer
     if (*abort) {  // let issued loads land before the CTA exits
       mbar_wait_drain(&bars[kBarQFull], 0);
       for (int c = issued - 1; c >= 0 && c >= issued - kStages; --c)
@@ -655,7 +756,7 @@ __device__ __forceinline__ void softmax_role(const TcParams& p, uint8_t* smem, u
 
 }
 
-template <int D>
+template <int D, bool G>
 __global__ void __launch_bounds__(kThreads, 1)
 at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
@@ -718,7 +819,8 @@ at_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorM
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(regs_low<D>()));
     if (warp == 0) {
-      producer_role<D>(tmQ, tmK, tmV, tmKc, tmVc, p, smem, h, a, row0, ntiles, lane, abort);
+      producer_role<D, G>(tmQ, tmK, tmV, tmKc, tmVc, p, smem, h, a, row0, ntiles,
+                          rows_a + rows_b, lane, abort);
     } else if (warp == 1) {
       mma_role<D>(p, smem, tmem, ntiles, abort);
     }
@@ -795,7 +897,7 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int box_r
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool G>
 ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_items,
                 uint16_t* kc16, uint16_t* vc16, int ck_pad, cudaStream_t s) {
   using L = Layout<D>;
@@ -804,8 +906,10 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
                                                                    a.c_k, ck_pad, D, total);
   EAR_TRY(after_launch());
   CUtensorMap mq, mk, mv, mkc, mvc;
-  if (!make_map(&mq, a.Q, a.bh * a.n_q, D, kTileRows) ||
-      !make_map(&mk, a.K, a.bh * a.n_k, D, kBox) || !make_map(&mv, a.V, a.bh * a.n_k, D, kBox) ||
+  // gather: one-row boxes (tile::gather4 fetches four of them per copy)
+  if (!make_map(&mq, a.Q, a.bh * a.n_q, D, G ? 1 : kTileRows) ||
+      !make_map(&mk, a.K, a.bh * a.n_k, D, G ? 1 : kBox) ||
+      !make_map(&mv, a.V, a.bh * a.n_k, D, G ? 1 : kBox) ||
       !make_map(&mkc, kc16, a.bh * ck_pad, D, kBox) ||
       !make_map(&mvc, vc16, a.bh * ck_pad, D, kBox))
     return EAR_ERR_CUDA;
@@ -813,6 +917,7 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
   p.q_off = a.q_off;
   p.k_off = a.k_off;
   p.q_perm = a.q_perm;
+  p.k_perm = a.k_perm;
   p.exact = a.exact;
   p.blk_off = a.blk_off;
   p.blk_list = a.blk_list;
@@ -829,14 +934,15 @@ ear_status tc_t(const AttnArgs& a, int2* items, int32_t* count, int64_t max_item
   p.O = static_cast<uint16_t*>(a.O);
   p.lse = a.lse;
   p.status = device_status_word();
-  EAR_CUDA(cudaFuncSetAttribute(at_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  EAR_CUDA(cudaFuncSetAttribute(at_tc<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kBytes));
   // setmaxnreg.inc waits until the block's launch registers cover the split:
   // refuse to launch a build whose allocation does not.
   cudaFuncAttributes fa;
-  EAR_CUDA(cudaFuncGetAttributes(&fa, at_tc<D>));
+  EAR_CUDA(cudaFuncGetAttributes(&fa, at_tc<D, G>));
   if (fa.numRegs * kThreads < 128 * regs_low<D>() + 256 * kRegsHigh) return EAR_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)max_items, (unsigned)a.bh);
-  at_tc<D><<<grid, kThreads, L::kBytes, s>>>(mq, mk, mv, mkc, mvc, p);
+  at_tc<D, G><<<grid, kThreads, L::kBytes, s>>>(mq, mk, mv, mkc, mvc, p);
   return after_launch();
 }
 
@@ -851,10 +957,16 @@ int64_t attention_tc_items_per_slice(int64_t n_q, int32_t c_q) {
 
 ear_status attention_tc_run(const AttnArgs& a, int2* items, int32_t* count, int64_t max_items,
                             uint16_t* kc16, uint16_t* vc16, cudaStream_t s) {
-  EAR_TRY(attention_plan(a.q_off, a.bh, a.c_q, kUnitRows, max_items, items, count, s));
   const int ck_pad = (int)attention_tc_ck_pad(a.c_k);
-  return a.d == 64 ? tc_t<64>(a, items, count, max_items, kc16, vc16, ck_pad, s)
-                   : tc_t<128>(a, items, count, max_items, kc16, vc16, ck_pad, s);
+  // TMA row coordinates are int32
+  if (a.bh * a.n_q > INT32_MAX || a.bh * a.n_k > INT32_MAX || a.bh * ck_pad > INT32_MAX)
+    return EAR_ERR_UNSUPPORTED;
+  EAR_TRY(attention_plan(a.q_off, a.bh, a.c_q, kUnitRows, max_items, items, count, s));
+  if (a.k_perm != nullptr)
+    return a.d == 64 ? tc_t<64, true>(a, items, count, max_items, kc16, vc16, ck_pad, s)
+                     : tc_t<128, true>(a, items, count, max_items, kc16, vc16, ck_pad, s);
+  return a.d == 64 ? tc_t<64, false>(a, items, count, max_items, kc16, vc16, ck_pad, s)
+                   : tc_t<128, false>(a, items, count, max_items, kc16, vc16, ck_pad, s);
 }
 
 }  // namespace ear

@@ -120,8 +120,9 @@ ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_
                              int32_t c, const void* X, void* X_perm, ear_dtype dtype, int32_t d,
                              float* seg_mean, void* stream) {
   if (bh < 1 || n < 1 || n > kMaxN || c < 1) return EAR_ERR_ARG;
-  if (!ok_ptr(perm) || !ok_ptr(offsets) || !ok_ptr(X) || !ok_ptr(X_perm) || !ok_dtype(dtype))
-    return EAR_ERR_ARG;
+  if (!ok_ptr(perm) || !ok_ptr(offsets) || !ok_ptr(X) || !ok_dtype(dtype)) return EAR_ERR_ARG;
+  // X_perm may be NULL only when the means are asked for (means only)
+  if (X_perm == nullptr ? seg_mean == nullptr : !ok_ptr(X_perm)) return EAR_ERR_ARG;
   if (seg_mean != nullptr && !aligned16(seg_mean)) return EAR_ERR_ARG;
   if (c > kMaxC || bh > kMaxBH || !ok_d(d)) return EAR_ERR_UNSUPPORTED;
   if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
@@ -129,12 +130,17 @@ ear_status ear_permute_apply(const int32_t* perm, const int32_t* offsets, int64_
                                 static_cast<cudaStream_t>(stream));
 }
 
-ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
-                     const float* k_centroids, const void* K_perm, ear_dtype dtype,
-                     const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V_perm,
-                     const float* v_centroids, float* E, void* ws, size_t ws_bytes,
-                     void* stream) {
+}  // extern "C"
+
+namespace {
+
+// ear_probe and ear_probe_gather: k_perm == nullptr means K / V are permuted.
+ear_status probe_entry(const float* q_centroids, const int32_t* q_counts,
+                       const float* k_centroids, const void* K_perm, const int32_t* k_perm,
+                       ear_dtype dtype, const int32_t* k_offsets, int64_t bh, int64_t n_k,
+                       int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                       const void* V_perm, const float* v_centroids, float* E, void* ws,
+                       size_t ws_bytes, void* stream) {
   if (!ok_dtype(dtype) || bh < 1 || n_k < 1 || n_k > kMaxN || c_q < 1 || c_k < 1 ||
       !std::isfinite(scale) || mode < EAR_PROBE_LOGIT || mode > EAR_PROBE_VALUE)
     return EAR_ERR_ARG;
@@ -146,9 +152,34 @@ ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
   if (mode != EAR_PROBE_LOGIT && dtype != EAR_BF16) return EAR_ERR_UNSUPPORTED;
   EAR_TRY(check_ws(ws, ws_bytes, ear::probe_workspace(bh, n_k, d, c_q, c_k)));
   if (ear::device_status_word() == nullptr) return EAR_ERR_CUDA;
-  return ear::probe_run(q_centroids, q_counts, k_centroids, K_perm, dtype, k_offsets, bh, n_k,
-                        d, c_q, c_k, scale, mode, V_perm, v_centroids, E, ws,
+  return ear::probe_run(q_centroids, q_counts, k_centroids, K_perm, k_perm, dtype, k_offsets, bh,
+                        n_k, d, c_q, c_k, scale, mode, V_perm, v_centroids, E, ws,
                         static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
+                     const float* k_centroids, const void* K_perm, ear_dtype dtype,
+                     const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
+                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V_perm,
+                     const float* v_centroids, float* E, void* ws, size_t ws_bytes,
+                     void* stream) {
+  return probe_entry(q_centroids, q_counts, k_centroids, K_perm, nullptr, dtype, k_offsets, bh,
+                     n_k, d, c_q, c_k, scale, mode, V_perm, v_centroids, E, ws, ws_bytes, stream);
+}
+
+ear_status ear_probe_gather(const float* q_centroids, const int32_t* q_counts,
+                            const float* k_centroids, const void* K, const int32_t* k_perm,
+                            ear_dtype dtype, const int32_t* k_offsets, int64_t bh, int64_t n_k,
+                            int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                            const void* V, const float* v_centroids, float* E, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (!ok_ptr(k_perm)) return EAR_ERR_ARG;
+  return probe_entry(q_centroids, q_counts, k_centroids, K, k_perm, dtype, k_offsets, bh, n_k, d,
+                     c_q, c_k, scale, mode, V, v_centroids, E, ws, ws_bytes, stream);
 }
 
 ear_status ear_route(const float* E, const int32_t* q_counts, const int32_t* k_counts,
@@ -241,14 +272,19 @@ ear_status ear_normalizer_change(const float* lse_sparse, const float* lse_dense
                                     static_cast<cudaStream_t>(stream));
 }
 
-ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_perm,
-                         ear_dtype dtype, const int32_t* q_offsets, const int32_t* k_offsets,
-                         const int32_t* q_perm, const float* k_centroids,
-                         const float* v_centroids, const uint8_t* exact,
-                         const int32_t* blk_offsets, const int32_t* blk_list, int64_t bh,
-                         int64_t n_q, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k,
-                         float scale, int32_t flags, void* O, float* lse, void* ws,
-                         size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// ear_attention and ear_attention_gather: k_perm == nullptr means Q / K / V are permuted.
+ear_status attention_entry(const void* Q_perm, const void* K_perm, const void* V_perm,
+                           ear_dtype dtype, const int32_t* q_offsets, const int32_t* k_offsets,
+                           const int32_t* q_perm, const int32_t* k_perm,
+                           const float* k_centroids, const float* v_centroids,
+                           const uint8_t* exact, const int32_t* blk_offsets,
+                           const int32_t* blk_list, int64_t bh, int64_t n_q, int64_t n_k,
+                           int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t flags,
+                           void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!ok_dtype(dtype) || bh < 1 || n_q < 1 || n_k < 1 || n_q > kMaxN || n_k > kMaxN ||
       c_q < 1 || c_k < 1 || !std::isfinite(scale) || (flags & ~EAR_COMPENSATE) != 0)
     return EAR_ERR_ARG;
@@ -263,7 +299,39 @@ ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_p
   ear::AttnArgs a{Q_perm, K_perm, V_perm, dtype, q_offsets, k_offsets, q_perm, k_centroids,
                   v_centroids, exact, blk_offsets, blk_list, bh, n_q, n_k, d, c_q, c_k, scale,
                   flags, O, lse};
+  a.k_perm = k_perm;
   return ear::attention_run(a, ws, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+ear_status ear_attention(const void* Q_perm, const void* K_perm, const void* V_perm,
+                         ear_dtype dtype, const int32_t* q_offsets, const int32_t* k_offsets,
+                         const int32_t* q_perm, const float* k_centroids,
+                         const float* v_centroids, const uint8_t* exact,
+                         const int32_t* blk_offsets, const int32_t* blk_list, int64_t bh,
+                         int64_t n_q, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k,
+                         float scale, int32_t flags, void* O, float* lse, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return attention_entry(Q_perm, K_perm, V_perm, dtype, q_offsets, k_offsets, q_perm, nullptr,
+                         k_centroids, v_centroids, exact, blk_offsets, blk_list, bh, n_q, n_k, d,
+                         c_q, c_k, scale, flags, O, lse, ws, ws_bytes, stream);
+}
+
+ear_status ear_attention_gather(const void* Q, const void* K, const void* V, ear_dtype dtype,
+                                const int32_t* q_offsets, const int32_t* k_offsets,
+                                const int32_t* q_perm, const int32_t* k_perm,
+                                const float* k_centroids, const float* v_centroids,
+                                const uint8_t* exact, const int32_t* blk_offsets,
+                                const int32_t* blk_list, int64_t bh, int64_t n_q, int64_t n_k,
+                                int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t flags,
+                                void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!ok_ptr(k_perm)) return EAR_ERR_ARG;
+  return attention_entry(Q, K, V, dtype, q_offsets, k_offsets, q_perm, k_perm, k_centroids,
+                         v_centroids, exact, blk_offsets, blk_list, bh, n_q, n_k, d, c_q, c_k,
+                         scale, flags, O, lse, ws, ws_bytes, stream);
 }
 
 ear_status ear_get_device_status(int32_t* out, void* stream) {

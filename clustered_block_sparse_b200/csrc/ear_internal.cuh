@@ -72,16 +72,17 @@ ear_status permute_apply_run(const int32_t* perm, const int32_t* offsets, int64_
                              float* seg_mean, cudaStream_t s);
 
 size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
-// Tensor-core probe (bf16 keys); mode as in ear_probe.
+// Tensor-core probe (bf16 keys); mode as in ear_probe.  kperm != nullptr:
+// K (and V) are in original order and permuted key j is row kperm[j].
 size_t probe_tc_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k);
 ear_status probe_tc_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                        const int32_t* koff, int64_t bh, int64_t n_k, int32_t d, int32_t c_q,
-                        int32_t c_k, float scale, int32_t mode, const void* V, const float* vc,
-                        float* E, void* ws, cudaStream_t s);
+                        const int32_t* kperm, const int32_t* koff, int64_t bh, int64_t n_k,
+                        int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                        const void* V, const float* vc, float* E, void* ws, cudaStream_t s);
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                     ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V,
-                     const float* vc, float* E, void* ws, cudaStream_t s);
+                     const int32_t* kperm, ear_dtype dt, const int32_t* koff, int64_t bh,
+                     int64_t n_k, int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                     const void* V, const float* vc, float* E, void* ws, cudaStream_t s);
 
 size_t route_workspace(int64_t bh, int32_t c_q, int32_t c_k);
 ear_status route_run(const float* E, const int32_t* qn, const int32_t* kn, int64_t bh,
@@ -128,6 +129,9 @@ struct AttnArgs {
   int32_t flags;
   void* O;
   float* lse;
+  // Gather: Q, K, V are in original token order and K / V rows are read as
+  // k_perm[r] (Q rows as q_perm[r]); nullptr = cluster-contiguous inputs.
+  const int32_t* k_perm = nullptr;
 };
 size_t attention_workspace(int64_t bh, int64_t n_q, int32_t d, int32_t c_q, int32_t c_k);
 ear_status attention_run(const AttnArgs& a, void* ws, cudaStream_t s);
@@ -147,6 +151,19 @@ ear_status attention_tc_run(const AttnArgs& a, int2* items, int32_t* count, int6
 namespace ear {
 
 __device__ __forceinline__ void latch(int* status, int code) { atomicCAS(status, 0, code); }
+
+// Gathered loads: the TMA row coordinate of original row perm[i] of slice h
+// (n rows per slice), or of the slice's row 0 with EAR_ERR_DEVICE latched when
+// the entry is out of range.
+__device__ __forceinline__ int32_t gather_row(const int32_t* perm, int64_t i, int64_t h,
+                                              int64_t n, int* status) {
+  int32_t o = perm[i];
+  if (o < 0 || o >= n) {
+    latch(status, EAR_ERR_DEVICE);
+    o = 0;
+  }
+  return (int32_t)(h * n) + o;
+}
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) {
   return __uint_as_float(static_cast<uint32_t>(u) << 16);

@@ -194,8 +194,9 @@ __device__ __forceinline__ void unpack16(const uint4 w, float (&f)[8], const flo
   for (int k = 4; k < 8; ++k) f[k] = 0.f;
 }
 
-// X_perm rows of cluster c = X[perm[r]] for r in [offsets[c], offsets[c+1]),
-// and their fp32 mean in a fixed order.  The offsets must partition [0, N)
+// X_perm rows of cluster c = X[perm[r]] for r in [offsets[c], offsets[c+1])
+// (skipped when Xp is null: the means alone), and their fp32 mean in a fixed
+// order.  The offsets must partition [0, N)
 // (offsets[0] = 0, offsets[C] = N, non-decreasing), as ear_permute writes
 // them; a table that does not is latched as an error.  A thread moves one
 // 16-byte piece of a row (kPer values) for every kGroups-th row of the
@@ -223,7 +224,7 @@ pm_gather_mean(const T* __restrict__ X, T* __restrict__ Xp, const int32_t* __res
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   const uint4* xh = reinterpret_cast<const uint4*>(X + h * N * D);
-  uint4* ph = reinterpret_cast<uint4*>(Xp + h * N * D);
+  uint4* ph = Xp != nullptr ? reinterpret_cast<uint4*>(Xp + h * N * D) : nullptr;
   const int32_t* pp = perm + h * N;
   for (int64_t r = r0 + g; r < r1; r += 2 * kGroups) {
     const int64_t ra = r, rb = r + kGroups;
@@ -236,13 +237,13 @@ pm_gather_mean(const T* __restrict__ X, T* __restrict__ Xp, const int32_t* __res
     if (okb) wb = xh[(int64_t)sb * kPieces + q];
     float f[8];
     if (oka) {
-      ph[ra * kPieces + q] = wa;
+      if (ph != nullptr) ph[ra * kPieces + q] = wa;
       unpack16(wa, f, X);
 #pragma unroll
       for (int k = 0; k < kPer; ++k) acc[k] += f[k];
     }
     if (okb) {
-      ph[rb * kPieces + q] = wb;
+      if (ph != nullptr) ph[rb * kPieces + q] = wb;
       unpack16(wb, f, X);
 #pragma unroll
       for (int k = 0; k < kPer; ++k) acc[k] += f[k];

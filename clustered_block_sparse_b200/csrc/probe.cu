@@ -37,8 +37,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
          const float* __restrict__ kc, const T* __restrict__ K,
-         const int32_t* __restrict__ koff, int64_t Nk, int Cq, int Ck, float scale,
-         float* __restrict__ E, int* status) {
+         const int32_t* __restrict__ kperm, const int32_t* __restrict__ koff, int64_t Nk, int Cq,
+         int Ck, float scale, float* __restrict__ E, int* status) {
   extern __shared__ float smem[];
   float* qs = smem;               // [D][kA]
   float* ks = qs + D * kA;        // [D][kJ]
@@ -80,8 +80,13 @@ pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
         for (int e = tid; e < kJ * (D / 4); e += kThreads) {
           const int j = e % kJ, k0 = (e / kJ) * 4;
           float v[4] = {0.f, 0.f, 0.f, 0.f};
-          if (j < nj) {
-            const int64_t base = (int64_t)(j0 + j) * D + k0;
+          // gather (kperm != nullptr): K in original order, permuted key r is row kperm[r]
+          const int64_t src = j >= nj ? -1
+                              : kperm == nullptr
+                                  ? (int64_t)(j0 + j)
+                                  : (int64_t)gather_row(kperm, h * Nk + j0 + j, h, Nk, status) - h * Nk;
+          if (src >= 0) {
+            const int64_t base = src * D + k0;
             float x[4];
             if constexpr (sizeof(T) == 2) {  // four bf16 in one 8-byte load
               const uint2 w = *reinterpret_cast<const uint2*>(kh + base);
@@ -157,13 +162,13 @@ pr_probe(const float* __restrict__ qc, const int32_t* __restrict__ qn,
 
 template <typename T, int D>
 ear_status run_t(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                 const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q, int32_t c_k,
-                 float scale, float* E, cudaStream_t s) {
+                 const int32_t* kperm, const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q,
+                 int32_t c_k, float scale, float* E, cudaStream_t s) {
   const size_t smem = ((size_t)(kA + kJ) * D + D) * sizeof(float);
   EAR_CUDA(cudaFuncSetAttribute(pr_probe<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem));
   pr_probe<T, D><<<dim3((unsigned)ceil_div(c_k, kClusters), (unsigned)bh), kThreads, smem, s>>>(
-      qc, qn, kc, (const T*)K, koff, n_k, c_q, c_k, scale, E, device_status_word());
+      qc, qn, kc, (const T*)K, kperm, koff, n_k, c_q, c_k, scale, E, device_status_word());
   return after_launch();
 }
 
@@ -177,13 +182,14 @@ size_t probe_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t 
 // The weight probes (mode 1, 2) are built for bf16 keys only (the ABI rejects
 // them for fp32 before this point).
 ear_status probe_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                     ear_dtype dt, const int32_t* koff, int64_t bh, int64_t n_k, int32_t d,
-                     int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V,
-                     const float* vc, float* E, void* ws, cudaStream_t s) {
+                     const int32_t* kperm, ear_dtype dt, const int32_t* koff, int64_t bh,
+                     int64_t n_k, int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                     const void* V, const float* vc, float* E, void* ws, cudaStream_t s) {
   if (dt == EAR_BF16)
-    return probe_tc_run(qc, qn, kc, K, koff, bh, n_k, d, c_q, c_k, scale, mode, V, vc, E, ws, s);
-  return d == 64 ? run_t<float, 64>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s)
-                 : run_t<float, 128>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, E, s);
+    return probe_tc_run(qc, qn, kc, K, kperm, koff, bh, n_k, d, c_q, c_k, scale, mode, V, vc, E,
+                        ws, s);
+  return d == 64 ? run_t<float, 64>(qc, qn, kc, K, kperm, koff, bh, n_k, c_q, c_k, scale, E, s)
+                 : run_t<float, 128>(qc, qn, kc, K, kperm, koff, bh, n_k, c_q, c_k, scale, E, s);
 }
 
 }  // namespace ear

@@ -15,7 +15,10 @@
 //             slice it touches, the WHOLE key clusters that start in its share
 //             (so every block sum is finished in one CTA, in a fixed order: E
 //             is deterministic); q̄ is reloaded when the slice changes.  A TMA warp
-//             streams 128-key tiles of K_perm; one elected thread issues
+//             streams 128-key tiles of K_perm (or, gathered, of K in original
+//             order: each lane looks up four rows' original indices in k_perm
+//             and the elected lane fetches them with tile::gather4 into the
+//             same swizzled tile); one elected thread issues
 //             tcgen05.mma (three MMAs per k step, one per q̄ part, fp32
 //             accumulation in TMEM, four accumulator buffers); four epilogue
 //             warps (one TMEM lane = one centroid row each) walk the tile's
@@ -61,7 +64,8 @@ struct PLayout {
   static constexpr int kBStage = kBHalf * (D / 64);
   static constexpr int kA = 0;
   static constexpr int kB = kA + kParts * kAPart;
-  static constexpr int kBar = kB + kStages * kBStage;
+  static constexpr int kGIdx = kB + kStages * kBStage;  // gather: one tile's row coordinates
+  static constexpr int kBar = kGIdx + kN * 4;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack to align the base to 1024
 };
@@ -71,6 +75,7 @@ struct PrParams {
   const int32_t* koff;    // [BH][C_k + 1]
   const float2* nmu;      // [BH][C_k][mtiles * kM]: -s μ as (hi, lo)
   float* E;               // [BH][C_q][C_k]
+  const int32_t* kperm;   // gather: original index of each permuted key; nullptr = K_perm given
   int64_t Nk;
   int Cq, Ck, mtiles;
   int64_t nseg;           // BH * mtiles segments of Nk key rows each
@@ -221,17 +226,40 @@ pr_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorM
       ++li;
       for (int i = 0; i < g.ntiles; ++i, ++t) {
         const int s = (int)(t % L::kStages);
+        int4 gi = make_int4(0, 0, 0, 0);
+        if (p.kperm != nullptr) {  // rows 4 lane .. 4 lane + 3 of the tile, looked up before the wait;
+                                   // rows past the segment repeat its last row
+          const int64_t kb = g.h * p.Nk;
+          const int32_t j = g.r0 + i * kN + 4 * lane, jl = g.r1 - 1;
+          gi.x = gather_row(p.kperm, kb + min(j, jl), g.h, p.Nk, p.status);
+          gi.y = gather_row(p.kperm, kb + min(j + 1, jl), g.h, p.Nk, p.status);
+          gi.z = gather_row(p.kperm, kb + min(j + 2, jl), g.h, p.Nk, p.status);
+          gi.w = gather_row(p.kperm, kb + min(j + 3, jl), g.h, p.Nk, p.status);
+        }
         if (t >= L::kStages &&
             !mbar_wait_warp(&bars[kBarBEmpty + s], (int)((t / L::kStages) - 1) & 1, abort)) {
           ok = false;
           break;
         }
-        if (leader) {
+        uint8_t* bdst = smem + L::kB + s * L::kBStage;
+        if (p.kperm != nullptr) {
+          int4* gidx = reinterpret_cast<int4*>(smem + L::kGIdx);
+          gidx[lane] = gi;
+          __syncwarp();
+          if (leader) {
+            mbar_arrive_expect_tx(&bars[kBarBFull + s], L::kBStage);
+            for (int q4 = 0; q4 < kN / 4; ++q4) {
+              const int4 rr = gidx[q4];
+              for (int hf = 0; hf < D / 64; ++hf)
+                tma_gather4(bdst + hf * L::kBHalf + q4 * 4 * 128, &tmK, &bars[kBarBFull + s],
+                            64 * hf, rr);
+            }
+          }
+        } else if (leader) {
           mbar_arrive_expect_tx(&bars[kBarBFull + s], L::kBStage);
           const int32_t row = (int32_t)(g.h * p.Nk + g.r0 + (int64_t)i * kN);
           for (int hf = 0; hf < D / 64; ++hf)
-            tma_load_2d(smem + L::kB + s * L::kBStage + hf * L::kBHalf, &tmK,
-                        &bars[kBarBFull + s], 64 * hf, row);
+            tma_load_2d(bdst + hf * L::kBHalf, &tmK, &bars[kBarBFull + s], 64 * hf, row);
         }
         __syncwarp();
       }
@@ -490,10 +518,12 @@ __global__ void pr_weigh(float* __restrict__ E, const float2* __restrict__ nmu,
 
 // Per permuted key j of cluster b: (|v_j - v̄_b|^2, (v_j - v̄_b)·v̄_b), and
 // |v̄_b|^2.  Block = (key cluster, slice); a warp per key row, lanes over d.
+// perm != nullptr: V is in original order and permuted row j is V[perm[j]].
 template <int D>
-__global__ void pr_vstats(const uint16_t* __restrict__ V, const float* __restrict__ vc,
-                          const int32_t* __restrict__ koff, int64_t Nk, int Ck,
-                          float2* __restrict__ vst, float* __restrict__ vnorm, int* status) {
+__global__ void pr_vstats(const uint16_t* __restrict__ V, const int32_t* __restrict__ perm,
+                          const float* __restrict__ vc, const int32_t* __restrict__ koff,
+                          int64_t Nk, int Ck, float2* __restrict__ vst,
+                          float* __restrict__ vnorm, int* status) {
   constexpr int kPer = D / 32;
   const int b = blockIdx.x;
   const int64_t h = blockIdx.y;
@@ -515,7 +545,8 @@ __global__ void pr_vstats(const uint16_t* __restrict__ V, const float* __restric
   for (int off = 16; off >= 1; off >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, off);
   if (threadIdx.x == 0) vnorm[h * Ck + b] = nv;
   for (int32_t j = r0 + w; j < r1; j += nw) {
-    const uint16_t* row = V + (h * Nk + j) * D + lane * kPer;
+    const int64_t src = perm != nullptr ? gather_row(perm, h * Nk + j, h, Nk, status) : h * Nk + j;
+    const uint16_t* row = V + src * D + lane * kPer;
     float uu = 0.f, uv = 0.f;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
@@ -587,7 +618,8 @@ PrWs carve(Carver& cv, int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32_t 
 
 template <int D, int MODE>
 ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                  const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q, int32_t c_k,
+                  const int32_t* kperm, const int32_t* koff, int64_t bh, int64_t n_k, int32_t c_q,
+                  int32_t c_k,
                   float scale, const void* V, const float* vc, float* E, void* ws,
                   cudaStream_t s) {
   using L = PLayout<D>;
@@ -604,7 +636,7 @@ ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const voi
   EAR_TRY(after_launch());
   CUtensorMap ma, mk;
   if (!make_map(&ma, w.qsplit, bh * mt * kParts * kM, D, kM) ||
-      !make_map(&mk, K, bh * n_k, D, kN))
+      !make_map(&mk, K, bh * n_k, D, kperm != nullptr ? 1 : kN))
     return EAR_ERR_CUDA;
   // Persistent: one CTA per SM (at most), each a contiguous share of the
   // (slice, M tile, key row) space, about 2048 key rows at least.
@@ -615,6 +647,7 @@ ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const voi
   p.koff = koff;
   p.nmu = w.nmu;
   p.E = E;
+  p.kperm = kperm;
   p.Nk = n_k;
   p.Cq = c_q;
   p.Ck = c_k;
@@ -628,7 +661,7 @@ ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const voi
   if (MODE > 0) EAR_CUDA(cudaMemsetAsync(w.zmax, 0, sizeof(uint32_t) * bh * mt * kM, s));
   if (MODE == 2) {
     pr_vstats<D><<<dim3((unsigned)c_k, (unsigned)bh), 128, 0, s>>>(
-        static_cast<const uint16_t*>(V), vc, koff, n_k, c_k, w.vst, w.vnorm, p.status);
+        static_cast<const uint16_t*>(V), kperm, vc, koff, n_k, c_k, w.vst, w.vnorm, p.status);
     EAR_TRY(after_launch());
   }
   EAR_CUDA(cudaFuncSetAttribute(pr_tc<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -652,10 +685,12 @@ size_t probe_tc_workspace(int64_t bh, int64_t n_k, int32_t d, int32_t c_q, int32
 }
 
 ear_status probe_tc_run(const float* qc, const int32_t* qn, const float* kc, const void* K,
-                        const int32_t* koff, int64_t bh, int64_t n_k, int32_t d, int32_t c_q,
-                        int32_t c_k, float scale, int32_t mode, const void* V, const float* vc,
-                        float* E, void* ws, cudaStream_t s) {
-#define EAR_PR(DD, MM) run_tc<DD, MM>(qc, qn, kc, K, koff, bh, n_k, c_q, c_k, scale, V, vc, E, ws, s)
+                        const int32_t* kperm, const int32_t* koff, int64_t bh, int64_t n_k,
+                        int32_t d, int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                        const void* V, const float* vc, float* E, void* ws, cudaStream_t s) {
+  if (bh * n_k > INT32_MAX) return EAR_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+#define EAR_PR(DD, MM) \
+  run_tc<DD, MM>(qc, qn, kc, K, kperm, koff, bh, n_k, c_q, c_k, scale, V, vc, E, ws, s)
   if (d == 64)
     return mode == 0 ? EAR_PR(64, 0) : mode == 1 ? EAR_PR(64, 1) : EAR_PR(64, 2);
   return mode == 0 ? EAR_PR(128, 0) : mode == 1 ? EAR_PR(128, 1) : EAR_PR(128, 2);

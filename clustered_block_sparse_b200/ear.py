@@ -92,16 +92,17 @@ def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor]
 
 
 def ear_permute_apply(perm: torch.Tensor, offsets: torch.Tensor, x: torch.Tensor,
-                      seg_mean: bool = False):
+                      seg_mean: bool = False, write_perm: bool = True):
     """X_perm[r] = X[perm[r]] with a permutation made by ear_permute, plus the
     optional per-cluster means (SVG-EAR §4.3: V in K's cluster order, v̄).
+    write_perm=False (with seg_mean) computes the means alone.
 
-    Returns (x_perm, mean [BH,C,d] f32 or None)."""
+    Returns (x_perm or None, mean [BH,C,d] f32 or None)."""
     for t, nm in ((perm, "perm"), (offsets, "offsets"), (x, "x")):
         _need(t, nm)
     bh, n, d = x.shape
     c = offsets.shape[1] - 1
-    x_perm = torch.empty_like(x)
+    x_perm = torch.empty_like(x) if write_perm else None
     mean = torch.empty((bh, c, d), dtype=torch.float32, device=x.device) if seg_mean else None
     N.check("ear_permute_apply", N.lib().ear_permute_apply(
         _p(perm), _p(offsets), bh, n, c, _p(x), _p(x_perm), _dtype(x), d, _p(mean),
@@ -156,6 +157,29 @@ def ear_probe(q_centroids, q_counts, k_centroids, k_perm, k_offsets, scale: Opti
         _p(q_centroids), _p(q_counts), _p(k_centroids), _p(k_perm), _dtype(k_perm), _p(k_offsets),
         bh, n_k, d, c_q, c_k, ctypes.c_float(s), int(mode), _p(v_perm), _p(v_centroids), _p(e),
         _p(ws), nb, _stream(k_perm.device)))
+    return e
+
+
+def ear_probe_gather(q_centroids, q_counts, k_centroids, k, k_perm_idx, k_offsets,
+                     scale: Optional[float] = None, mode: int = 0, v=None, v_centroids=None):
+    """ear_probe on keys (and values) in their original order: permuted key r is
+    k[k_perm_idx[r]].  Same E as ear_probe(..., k[k_perm_idx], ...)."""
+    for t, nm in ((q_centroids, "q_centroids"), (q_counts, "q_counts"), (k_centroids, "k_centroids"),
+                  (k, "k"), (k_perm_idx, "k_perm_idx"), (k_offsets, "k_offsets")):
+        _need(t, nm)
+    if mode == N.EAR_PROBE_VALUE:
+        _need(v, "v")
+        _need(v_centroids, "v_centroids")
+    bh, c_q, d = q_centroids.shape
+    c_k = k_centroids.shape[1]
+    n_k = k.shape[1]
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    e = torch.empty((bh, c_q, c_k), dtype=torch.float32, device=k.device)
+    ws, nb = _workspace(N.EAR_OP_PROBE, bh, 0, n_k, d, c_q, c_k, k.device)
+    N.check("ear_probe_gather", N.lib().ear_probe_gather(
+        _p(q_centroids), _p(q_counts), _p(k_centroids), _p(k), _p(k_perm_idx), _dtype(k),
+        _p(k_offsets), bh, n_k, d, c_q, c_k, ctypes.c_float(s), int(mode), _p(v), _p(v_centroids),
+        _p(e), _p(ws), nb, _stream(k.device)))
     return e
 
 
@@ -282,6 +306,31 @@ def ear_attention(q_perm_x, k_perm_x, v_perm_x, q_offsets, k_offsets, q_perm, k_
     return o, lse
 
 
+def ear_attention_gather(q, k, v, q_offsets, k_offsets, q_perm, k_perm_idx, k_centroids,
+                         v_centroids, exact, blk_offsets, blk_list, scale: Optional[float] = None,
+                         compensate: bool = True, want_lse: bool = False,
+                         out: Optional[torch.Tensor] = None):
+    """ear_attention on q, k, v in their original order (the permutation folded
+    into the loads): permuted query r is q[q_perm[r]], permuted key r is
+    k[k_perm_idx[r]] / v[k_perm_idx[r]].  Same O and lse as ear_attention on the
+    permuted copies."""
+    bh, n_q, d = q.shape
+    n_k = k.shape[1]
+    c_q = q_offsets.shape[1] - 1
+    c_k = k_offsets.shape[1] - 1
+    dev = q.device
+    s = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((bh, n_q), dtype=torch.float32, device=dev) if want_lse else None
+    ws, nb = _workspace(N.EAR_OP_ATTENTION, bh, n_q, n_k, d, c_q, c_k, dev)
+    N.check("ear_attention_gather", N.lib().ear_attention_gather(
+        _p(q), _p(k), _p(v), _dtype(q), _p(q_offsets), _p(k_offsets), _p(q_perm), _p(k_perm_idx),
+        _p(k_centroids), _p(v_centroids), _p(exact), _p(blk_offsets), _p(blk_list),
+        bh, n_q, n_k, d, c_q, c_k, ctypes.c_float(s), N.EAR_COMPENSATE if compensate else 0,
+        _p(o), _p(lse), _p(ws), nb, _stream(dev)))
+    return o, lse
+
+
 def ear_selftest_wait_timeout(device=None) -> None:
     """Enqueue the bounded-wait self-test: the next ear_get_device_status() on
     this device reports EAR_ERR_TIMEOUT (after about one second)."""
@@ -321,16 +370,30 @@ class LayerResult:
 
 def ear_layer(q, k, v, q_init, k_init, iters: int, density: float, ratio_mode: int = 0,
               compensate: bool = True, want_lse: bool = False, scale: Optional[float] = None,
-              out: Optional[torch.Tensor] = None) -> LayerResult:
-    """One SVG-EAR attention layer: the five entry points in order (SVG-EAR §3.1, §4)."""
+              out: Optional[torch.Tensor] = None, gather: bool = False) -> LayerResult:
+    """One SVG-EAR attention layer: the five entry points in order (SVG-EAR §3.1, §4).
+
+    gather=True keeps Q, K and V in their original order: the permutations are
+    computed but never applied to a copy; the probe and the attention read rows
+    through them (same results)."""
     n_q, n_k = q.shape[1], k.shape[1]
     qc, ql, qn = ear_kmeans(q, q_init, iters)
     kc, kl, kn = ear_kmeans(k, k_init, iters)
-    qp, qo, qx, _ = ear_permute(ql, q_init.shape[1], q)
-    kp, ko, kx, _ = ear_permute(kl, k_init.shape[1], k)
-    vx, vm = ear_permute_apply(kp, ko, v, seg_mean=True)
-    e = ear_probe(qc, qn, kc, kx, ko, scale)
+    if gather:
+        qp, qo, _, _ = ear_permute(ql, q_init.shape[1])
+        kp, ko, _, _ = ear_permute(kl, k_init.shape[1])
+        _, vm = ear_permute_apply(kp, ko, v, seg_mean=True, write_perm=False)
+        e = ear_probe_gather(qc, qn, kc, k, kp, ko, scale)
+    else:
+        qp, qo, qx, _ = ear_permute(ql, q_init.shape[1], q)
+        kp, ko, kx, _ = ear_permute(kl, k_init.shape[1], k)
+        vx, vm = ear_permute_apply(kp, ko, v, seg_mean=True)
+        e = ear_probe(qc, qn, kc, kx, ko, scale)
     exact, bo, bl, pairs = ear_route(e, qn, kn, n_q, n_k, density, ratio_mode)
-    o, lse = ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, scale, compensate,
-                           want_lse, out)
+    if gather:
+        o, lse = ear_attention_gather(q, k, v, qo, ko, qp, kp, kc, vm, exact, bo, bl, scale,
+                                      compensate, want_lse, out)
+    else:
+        o, lse = ear_attention(qx, kx, vx, qo, ko, qp, kc, vm, exact, bo, bl, scale, compensate,
+                               want_lse, out)
     return LayerResult(o, lse, qc, ql, qn, kc, kl, kn, qp, qo, kp, ko, vm, e, exact, bo, bl, pairs)

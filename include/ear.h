@@ -14,6 +14,10 @@
  *   ear_route                          greedy error-to-cost block selection
  *   ear_attention                      block-sparse exact attention plus
  *                                      centroid compensation, one softmax
+ * or, with no permuted copy of Q, K or V (the gathered layer):
+ *   ear_kmeans(Q), ear_kmeans(K); ear_permute(Q), (K) without X (perm and
+ *   offsets only); ear_permute_apply(V, K's perm) with X_perm = NULL (v̄
+ *   only); ear_probe_gather; ear_route; ear_attention_gather.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -142,7 +146,9 @@ EAR_API ear_status ear_permute(const int32_t* labels, int64_t bh, int64_t n, int
  *   perm     [BH][N] int32          from ear_permute (a bijection of [0, N))
  *   offsets  [BH][C+1] int32        from the same call
  *   X        [BH][N][d] dtype       rows in original order
- *   X_perm   [BH][N][d] dtype  out  X_perm[r] = X[perm[r]]
+ *   X_perm   [BH][N][d] dtype  out  X_perm[r] = X[perm[r]]; may be NULL when
+ *                                   seg_mean is given (the means alone: the
+ *                                   gathered layer keeps V in original order)
  *   seg_mean [BH][C][d] float  out  optional mean of X's rows of each cluster
  *                                   (rows offsets[c] .. offsets[c+1]-1 of
  *                                   X_perm); zero rows for empty clusters
@@ -218,6 +224,26 @@ EAR_API ear_status ear_probe(const float* q_centroids, const int32_t* q_counts,
                      int32_t c_q, int32_t c_k, float scale, int32_t mode, const void* V_perm,
                      const float* v_centroids, float* E, void* ws, size_t ws_bytes,
                      void* stream);
+
+/*
+ * ear_probe on keys (and values) left in their ORIGINAL token order (SVG-EAR
+ * §3.1's cluster-contiguous layout folded into the loads, no permuted copy):
+ *   K        [BH][N_k][d] dtype   keys in original order
+ *   k_perm   [BH][N_k] int32      from ear_permute of K's labels: permuted
+ *                                 key r is K[k_perm[r]]
+ *   V        [BH][N_k][d] dtype   values in original order (EAR_PROBE_VALUE; else NULL)
+ * Every other argument, the workspace (EAR_OP_PROBE) and E are as in
+ * ear_probe, whose result this reproduces bit for bit on K_perm = K[k_perm].
+ * A k_perm entry outside [0, N_k) latches EAR_ERR_DEVICE and row 0 is read
+ * in its place.
+ */
+EAR_API ear_status ear_probe_gather(const float* q_centroids, const int32_t* q_counts,
+                                    const float* k_centroids, const void* K,
+                                    const int32_t* k_perm, ear_dtype dtype,
+                                    const int32_t* k_offsets, int64_t bh, int64_t n_k, int32_t d,
+                                    int32_t c_q, int32_t c_k, float scale, int32_t mode,
+                                    const void* V, const float* v_centroids, float* E, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /*
  * Greedy error-to-cost routing under a density budget (SVG-EAR §4.2 "Error
@@ -314,6 +340,32 @@ EAR_API ear_status ear_attention(const void* Q_perm, const void* K_perm, const v
                          int64_t n_q, int64_t n_k, int32_t d, int32_t c_q, int32_t c_k,
                          float scale, int32_t flags, void* O, float* lse, void* ws,
                          size_t ws_bytes, void* stream);
+
+/*
+ * ear_attention on Q, K and V left in their ORIGINAL token order (SVG-EAR
+ * §3.1's cluster-contiguous layout folded into the loads: bf16 rows are
+ * fetched four at a time with TMA tile::gather4, so no permuted copy of Q,
+ * K or V is ever written).
+ *   Q        [BH][N_q][d] dtype   queries in original order
+ *   K, V     [BH][N_k][d] dtype   keys and values in original order
+ *   q_perm   [BH][N_q] int32      permuted query r is Q[q_perm[r]] (and its
+ *                                 output row is O[q_perm[r]], as in ear_attention)
+ *   k_perm   [BH][N_k] int32      permuted key r is K[k_perm[r]], V[k_perm[r]]
+ * Every other argument, the workspace (EAR_OP_ATTENTION), O and lse are as in
+ * ear_attention, whose result this reproduces bit for bit on
+ * Q_perm = Q[q_perm], K_perm = K[k_perm], V_perm = V[k_perm].  A k_perm entry
+ * outside [0, N_k) latches EAR_ERR_DEVICE and row 0 is read in its place.
+ */
+EAR_API ear_status ear_attention_gather(const void* Q, const void* K, const void* V,
+                                        ear_dtype dtype, const int32_t* q_offsets,
+                                        const int32_t* k_offsets, const int32_t* q_perm,
+                                        const int32_t* k_perm, const float* k_centroids,
+                                        const float* v_centroids, const uint8_t* exact,
+                                        const int32_t* blk_offsets, const int32_t* blk_list,
+                                        int64_t bh, int64_t n_q, int64_t n_k, int32_t d,
+                                        int32_t c_q, int32_t c_k, float scale, int32_t flags,
+                                        void* O, float* lse, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /*
  * Clustering diagnostics (SVG-EAR §4.2: the error bound's residual

@@ -95,6 +95,24 @@ def test_permute_apply_validation(lib):
     assert f(FAKE, FAKE, 1, 100, 4, None, FAKE, 1, 128, None, None) == N.EAR_ERR_ARG
     assert f(FAKE, FAKE, 1, 100, 4, FAKE, FAKE, 1, 128, MISALIGNED, None) == N.EAR_ERR_ARG
     assert f(FAKE, FAKE, 1, 100, 4, FAKE, FAKE, 1, 96, None, None) == N.EAR_ERR_UNSUPPORTED
+    # X_perm may be left out only when the means are asked for
+    assert f(FAKE, FAKE, 1, 100, 4, FAKE, None, 1, 128, None, None) == N.EAR_ERR_ARG
+    assert f(FAKE, FAKE, 1, 100, 4, FAKE, None, 1, 96, FAKE, None) == N.EAR_ERR_UNSUPPORTED
+
+
+def test_probe_gather_validation(lib):
+    f = lib.ear_probe_gather
+
+    def call(K=FAKE, kp=FAKE, d=128, mode=0, V=None, vc=None):
+        return f(FAKE, FAKE, FAKE, K, kp, 1, FAKE, 1, 100, d, 4, 4, ctypes.c_float(0.1), mode, V,
+                 vc, FAKE, None, 0, None)
+    assert call(kp=None) == N.EAR_ERR_ARG
+    assert call(kp=MISALIGNED) == N.EAR_ERR_ARG
+    assert call(K=None) == N.EAR_ERR_ARG
+    assert call(mode=3) == N.EAR_ERR_ARG
+    assert call(mode=N.EAR_PROBE_VALUE) == N.EAR_ERR_ARG          # values missing
+    assert call(d=32) == N.EAR_ERR_UNSUPPORTED
+    assert call(mode=N.EAR_PROBE_VALUE, V=FAKE, vc=FAKE, d=32) == N.EAR_ERR_UNSUPPORTED
 
 
 def test_probe_validation(lib):
@@ -130,6 +148,19 @@ def test_attention_validation(lib):
     assert call(flags=4) == N.EAR_ERR_ARG
     assert call(lse=MISALIGNED) == N.EAR_ERR_ARG
     assert call(scale=float("inf")) == N.EAR_ERR_ARG
+    assert call(d=256) == N.EAR_ERR_UNSUPPORTED
+
+
+def test_attention_gather_validation(lib):
+    f = lib.ear_attention_gather
+
+    def call(kp=FAKE, flags=1, d=128, Q=FAKE):
+        return f(Q, FAKE, FAKE, 1, FAKE, FAKE, FAKE, kp, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 100, 100,
+                 d, 4, 4, ctypes.c_float(0.1), flags, FAKE, None, FAKE, 1 << 30, None)
+    assert call(kp=None) == N.EAR_ERR_ARG
+    assert call(kp=MISALIGNED) == N.EAR_ERR_ARG
+    assert call(Q=None) == N.EAR_ERR_ARG
+    assert call(flags=4) == N.EAR_ERR_ARG
     assert call(d=256) == N.EAR_ERR_UNSUPPORTED
 
 
