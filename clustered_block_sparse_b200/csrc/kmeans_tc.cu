@@ -16,7 +16,10 @@
 //                streams X tiles, one thread issues tcgen05.mma
 //                (S = X C^T, fp32, 256-column chunks, two TMEM buffers) and
 //                two epilogue warpgroups scan each chunk (alternate 32-column
-//                groups) twice: pass 1 takes the minimum of
+//                groups; with one chunk per tile and one pass, C <= 256,
+//                alternate tiles instead, one TMEM buffer each, so two tiles
+//                are decided at once and no merge is needed) twice: pass 1
+//                takes the minimum of
 //                d~_c = ||c||^2 - 2 x.c^, pass 2 collects every column within
 //                the rounding margin of the running minimum.  Each warpgroup
 //                keeps its four best candidates by distance and the smallest
@@ -187,7 +190,9 @@ __device__ __forceinline__ uint32_t group_hits(const uint32_t (&v)[32], const fl
   return hit;
 }
 
-template <int D>
+// TP: tile-parallel epilogue (one 256-column chunk per tile and one pass:
+// the launcher picks it only then).
+template <int D, bool TP>
 __global__ void __launch_bounds__(kThreads, 1)
 km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
       const KmTcParams p, int* status) {
@@ -202,6 +207,13 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
   const int ntiles = (int)(left < kTilesPerCta ? left : kTilesPerCta);
   if (ntiles <= 0) return;
   const int nch = (p.cp_pass + kColChunk - 1) / kColChunk;
+  // tile-parallel epilogue: each warpgroup decides every other tile on its own
+  constexpr bool tp = TP;
+  constexpr int kNg = TP ? 8 : 4;  // column groups of a chunk one warpgroup scans
+  if (TP && (nch != 1 || p.carry_in || p.carry_out)) {
+    if (threadIdx.x == 0) latch(status, EAR_ERR_DEVICE);
+    return;
+  }
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -218,7 +230,7 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
     mbar_init(&bars[kBarDrain], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[kBarTmFull + b], 1);
-      mbar_init(&bars[kBarTmEmpty + b], 256);
+      mbar_init(&bars[kBarTmEmpty + b], tp ? 128 : 256);
     }
     *abort = 0;
     fence_barrier_init();
@@ -317,18 +329,26 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
     bool ok = true;
     // ||x|| and the old label of the next tile's row are loaded a tile ahead
     auto row_of = [&](int t) { return (tile0 + t) * kTileRows + r; };
-    float xn_next = row_of(0) < p.N ? p.xnorm[h * p.N + row_of(0)] : 0.f;
-    int old_next = (w == 0 && !p.first && row_of(0) < p.N) ? p.labels[h * p.N + row_of(0)] : -1;
-    for (int t = 0; t < ntiles; ++t) {
+    // tp: this warpgroup's tiles are w, w + 2, ...; it decides them alone
+    const int t_first = tp ? w : 0, t_step = tp ? 2 : 1;
+    const bool decider = tp || w == 0;
+    float xn_next = 0.f;
+    int old_next = -1;
+    if (t_first < ntiles) {
+      const int64_t r0 = row_of(t_first);
+      xn_next = r0 < p.N ? p.xnorm[h * p.N + r0] : 0.f;
+      old_next = (decider && !p.first && r0 < p.N) ? p.labels[h * p.N + r0] : -1;
+    }
+    for (int t = t_first; t < ntiles; t += t_step) {
       const int64_t row = row_of(t);
       const bool valid = row < p.N;
       const int64_t g = h * p.N + row;
       const float xn = xn_next;
       const int old_pre = old_next;
-      if (t + 1 < ntiles) {
-        const int64_t rn = row_of(t + 1);
+      if (t + t_step < ntiles) {
+        const int64_t rn = row_of(t + t_step);
         xn_next = rn < p.N ? p.xnorm[h * p.N + rn] : 0.f;
-        old_next = (w == 0 && !p.first && rn < p.N) ? p.labels[h * p.N + rn] : -1;
+        old_next = (decider && !p.first && rn < p.N) ? p.labels[h * p.N + rn] : -1;
       }
       const float margin =
           2.f * (p.a_coef * xn * cmax + p.b_coef * cmax * cmax + p.s_coef * (xn + cmax));
@@ -356,31 +376,35 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         tc_fence_after();
         const int n = min(kColChunk, p.cp_pass - j * kColChunk);
         const uint32_t tbuf = tmem + lane_bits + b * kColChunk;
-        // This warpgroup's column groups of the chunk: gg = w + 2u, u = 0..3.
+        // This warpgroup's column groups of the chunk: gg = w + 2u, u = 0..3
+        // (tp: all eight, gg = u).
         // Pass 1: minimum of each group (two groups per TMEM wait, four
         // independent min chains).  Columns past C_pad see cn = +inf; stale
         // TMEM there turns into +inf or NaN, and NaN never wins a comparison.
-        float gmin[4];
+        float gmin[kNg];
 #pragma unroll
-        for (int u = 0; u < 4; u += 2) {
-          const int ga = w + 2 * u, gb = w + 2 * (u + 1);
+        for (int u = 0; u < kNg; u += 2) {
+          gmin[u] = inf;
+          gmin[u + 1] = inf;
+          const int ga = tp ? u : w + 2 * u, gb = tp ? u + 1 : w + 2 * (u + 1);
           uint32_t va[32], vb[32];
           const bool has_a = ga * 32 < n, has_b = gb * 32 < n;
           if (has_a) tmem_ld32(tbuf + 32 * ga, va);
           if (has_b) tmem_ld32(tbuf + 32 * gb, vb);
           tmem_ld_wait();
-          gmin[u] = inf;
-          gmin[u + 1] = inf;
           if (has_a) gmin[u] = group_min(va, cn + j * kColChunk + 32 * ga);
           if (has_b) gmin[u + 1] = group_min(vb, cn + j * kColChunk + 32 * gb);
         }
-        run = fminf(run, fminf(fminf(gmin[0], gmin[1]), fminf(gmin[2], gmin[3])));
+        float gm = fminf(fminf(gmin[0], gmin[1]), fminf(gmin[2], gmin[3]));
+        if (TP) gm = fminf(gm, fminf(fminf(gmin[kNg - 4], gmin[kNg - 3]),
+                                     fminf(gmin[kNg - 2], gmin[kNg - 1])));
+        run = fminf(run, gm);
         // Pass 2: only groups whose minimum lies within the margin of the
         // running minimum can hold candidates (usually one group).
         const float thr = run + margin;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int gg = w + 2 * u;
+        for (int u = 0; u < kNg; ++u) {
+          const int gg = tp ? u : w + 2 * u;
           if (!__any_sync(0xffffffffu, gmin[u] <= thr)) continue;  // warp-uniform: tcgen05.ld
           uint32_t v[32];
           tmem_ld32(tbuf + 32 * gg, v);
@@ -407,26 +431,30 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         mbar_arrive(&bars[kBarTmEmpty + b]);
       }
       const int xo = (t & 1) * kTileRows + r;
-      if (w == 1) {
+      if (w == 1 && !tp) {
         xrun[xo] = run;
         reinterpret_cast<float*>(xcnt)[xo] = dropped;
         xcand[4 * xo + 0] = c0; xcand[4 * xo + 1] = c1; xcand[4 * xo + 2] = c2; xcand[4 * xo + 3] = c3;
         xdist[4 * xo + 0] = d0; xdist[4 * xo + 1] = d1; xdist[4 * xo + 2] = d2; xdist[4 * xo + 3] = d3;
       }
-      named_bar(1, 256);
-      if (w == 0 && ok && valid) {
+      if (!tp) named_bar(1, 256);
+      if (decider && ok && valid) {
         // this warpgroup's list, the other warpgroup's, and (after the first
         // pass) the state earlier passes carried for the row
-        float best = fminf(run, xrun[xo]);
-        float drop = fminf(dropped, reinterpret_cast<const float*>(xcnt)[xo]);
+        float best = run;
+        float drop = dropped;
         int cs[12];
         float ds[12];
         cs[0] = c0; cs[1] = c1; cs[2] = c2; cs[3] = c3;
         ds[0] = d0; ds[1] = d1; ds[2] = d2; ds[3] = d3;
+        if (!tp) {  // the other warpgroup's list
+          best = fminf(run, xrun[xo]);
+          drop = fminf(dropped, reinterpret_cast<const float*>(xcnt)[xo]);
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          cs[4 + u] = xcand[4 * xo + u];
-          ds[4 + u] = xdist[4 * xo + u];
+          cs[4 + u] = tp ? -1 : xcand[4 * xo + u];
+          ds[4 + u] = tp ? inf : xdist[4 * xo + u];
           cs[8 + u] = -1;
           ds[8 + u] = inf;
         }
@@ -901,7 +929,10 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
   // centroid values in the fp16 subnormal range round with absolute error
   // <= 2^-25: at most sqrt(d) 2^-25 ||x|| on x.c, doubled in d~
   p.s_coef = (float)(2.0 * std::sqrt((double)D) * std::ldexp(1.0, -25) * 1.01);
-  EAR_CUDA(cudaFuncSetAttribute(km_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  EAR_CUDA(cudaFuncSetAttribute(km_tc<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kBytes));
+  EAR_CUDA(cudaFuncSetAttribute(km_tc<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                L::kBytes));
   const dim3 grid((unsigned)ceil_div(ceil_div(n, kTileRows), kTilesPerCta), (unsigned)bh);
   const int64_t crow = bh * (int64_t)c;
   for (int t = 0; t < iters; ++t) {
@@ -911,7 +942,10 @@ ear_status run_tc(const uint16_t* X, int64_t bh, int64_t n, int32_t c, int32_t i
       p.cp_pass = std::min(kMaxCPad, cp - p.c0);
       p.carry_in = pass > 0 ? 1 : 0;
       p.carry_out = pass + 1 < npass ? 1 : 0;
-      km_tc<D><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
+      if (npass == 1 && cp <= kColChunk)  // one chunk per tile: tile-parallel epilogue
+        km_tc<D, true><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
+      else
+        km_tc<D, false><<<grid, kThreads, L::kBytes, s>>>(mx, mc, p, status);
       EAR_TRY(after_launch());
     }
     km_resolve<uint16_t, D><<<rgrid, 256, 0, s>>>(X, cent, n, c, rows, labels, p.first, w.kind,
