@@ -18,10 +18,11 @@
 //                two epilogue warpgroups scan each chunk (alternate 32-column
 //                groups; with one chunk per tile and one pass, C <= 256,
 //                alternate tiles instead, one TMEM buffer each, so two tiles
-//                are decided at once and no merge is needed) twice: pass 1
-//                takes the minimum of
-//                d~_c = ||c||^2 - 2 x.c^, pass 2 collects every column within
-//                the rounding margin of the running minimum.  Each warpgroup
+//                are decided at once and no merge is needed) in one pass:
+//                the minimum of d~_c = ||c||^2 - 2 x.c^ is taken group by
+//                group, and a group whose minimum lies within the rounding
+//                margin of the running minimum is searched for candidates
+//                from the same registers.  Each warpgroup
 //                keeps its four best candidates by distance and the smallest
 //                distance it had to drop.  One candidate within the margin of
 //                the row's minimum = a certain label; 2-4 go to an fp64
@@ -377,55 +378,44 @@ km_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorM
         const int n = min(kColChunk, p.cp_pass - j * kColChunk);
         const uint32_t tbuf = tmem + lane_bits + b * kColChunk;
         // This warpgroup's column groups of the chunk: gg = w + 2u, u = 0..3
-        // (tp: all eight, gg = u).
-        // Pass 1: minimum of each group (two groups per TMEM wait, four
-        // independent min chains).  Columns past C_pad see cn = +inf; stale
-        // TMEM there turns into +inf or NaN, and NaN never wins a comparison.
-        float gmin[kNg];
+        // (tp: all eight, gg = u), two per TMEM wait, each minimum in four
+        // independent chains.  Columns past C_pad see cn = +inf; stale TMEM
+        // there turns into +inf or NaN, and NaN never wins a comparison.
+        // One pass: each pair of groups is read from TMEM once; the running
+        // minimum moves group by group and a group whose minimum lies within
+        // the margin of it is searched for candidates from the same registers
+        // (the running threshold is never below the row's final minimum +
+        // margin, so every final candidate is inserted or counted as dropped).
+        auto scan = [&](const uint32_t (&v)[32], float gm, int gg) {
+          run = fminf(run, gm);
+          const float thr = run + margin;
+          if (!__any_sync(0xffffffffu, gm <= thr)) return;
+          if (gm > thr) return;
+          const int cbase = j * kColChunk + 32 * gg;
+          uint32_t hit = group_hits(v, cn + cbase, thr);
+          if ((hit & (hit - 1)) == 0) {
+            if (hit) insert(p.c0 + cbase + __ffs(hit) - 1, gm);
+            hit = 0;
+          }
+          while (hit) {
+            const int k = __ffs(hit) - 1;
+            hit &= hit - 1;
+            uint32_t vk = 0;
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) vk = kk == k ? v[kk] : vk;
+            insert(p.c0 + cbase + k, fmaf(-2.f, __uint_as_float(vk), cn[cbase + k]));
+          }
+        };
 #pragma unroll
         for (int u = 0; u < kNg; u += 2) {
-          gmin[u] = inf;
-          gmin[u + 1] = inf;
           const int ga = tp ? u : w + 2 * u, gb = tp ? u + 1 : w + 2 * (u + 1);
           uint32_t va[32], vb[32];
           const bool has_a = ga * 32 < n, has_b = gb * 32 < n;
           if (has_a) tmem_ld32(tbuf + 32 * ga, va);
           if (has_b) tmem_ld32(tbuf + 32 * gb, vb);
           tmem_ld_wait();
-          if (has_a) gmin[u] = group_min(va, cn + j * kColChunk + 32 * ga);
-          if (has_b) gmin[u + 1] = group_min(vb, cn + j * kColChunk + 32 * gb);
-        }
-        float gm = fminf(fminf(gmin[0], gmin[1]), fminf(gmin[2], gmin[3]));
-        if (TP) gm = fminf(gm, fminf(fminf(gmin[kNg - 4], gmin[kNg - 3]),
-                                     fminf(gmin[kNg - 2], gmin[kNg - 1])));
-        run = fminf(run, gm);
-        // Pass 2: only groups whose minimum lies within the margin of the
-        // running minimum can hold candidates (usually one group).
-        const float thr = run + margin;
-#pragma unroll
-        for (int u = 0; u < kNg; ++u) {
-          const int gg = tp ? u : w + 2 * u;
-          if (!__any_sync(0xffffffffu, gmin[u] <= thr)) continue;  // warp-uniform: tcgen05.ld
-          uint32_t v[32];
-          tmem_ld32(tbuf + 32 * gg, v);
-          tmem_ld_wait();
-          if (gmin[u] > thr) continue;
-          const int cbase = j * kColChunk + 32 * gg;  // column of this pass
-          uint32_t hit = group_hits(v, cn + cbase, thr);
-          if ((hit & (hit - 1)) == 0) {
-            // one hit (the usual case): it is the group's minimum column, so
-            // its d~ is gmin[u] and needs no extraction from v
-            if (hit) insert(p.c0 + cbase + __ffs(hit) - 1, gmin[u]);
-            hit = 0;
-          }
-          while (hit) {
-            const int k = __ffs(hit) - 1;
-            hit &= hit - 1;
-            uint32_t vk = 0;  // v[k] with a static index, so v stays in registers
-#pragma unroll
-            for (int kk = 0; kk < 32; ++kk) vk = kk == k ? v[kk] : vk;
-            insert(p.c0 + cbase + k, fmaf(-2.f, __uint_as_float(vk), cn[cbase + k]));
-          }
+          if (has_a) scan(va, group_min(va, cn + j * kColChunk + 32 * ga), ga);
+          if (has_b) scan(vb, group_min(vb, cn + j * kColChunk + 32 * gb), gb);
         }
         tc_fence_before();
         mbar_arrive(&bars[kBarTmEmpty + b]);
