@@ -204,7 +204,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/layer",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": value,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, args.gpus, args.layout),
+        "data": "synthetic", "config": config_of(w, args.gpus, args.layout, args.kmeans_streams),
         "cpu_baseline": {"value": value, "unit": "ms/layer", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "ms/layer", "h2d_bytes_per_step": 0,
@@ -233,10 +233,11 @@ def recorded_traffic(heads: int):
     return per_head * heads if sha == cur else None
 
 
-def config_of(w, n_gpus, layout="permuted"):
+def config_of(w, n_gpus, layout="permuted", kmeans_streams=2):
     return {"workload": w.name, "heads": w.heads, "n_q": w.n, "n_k": w.n, "d": w.d,
             "c_q": w.c_q, "c_k": w.c_k, "kmeans_iters": w.iters, "density": w.density,
             "ratio_mode": 0, "compensate": True,
+            "kmeans_streams": kmeans_streams,
             "layout": ("gathered: Q, K, V stay in token order; probe and attention read rows "
                        "through the permutations (TMA tile::gather4)" if layout == "gathered"
                        else "permuted: cluster-contiguous copies of Q, K, V"),
@@ -285,8 +286,8 @@ def run_ear(args, w):
         """One layer; `ev` = 6 events recorded at the stage boundaries."""
         rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
         rec(0)
-        qc, ql, qn = ear.ear_kmeans(q, qi, w.iters)
-        kc, kl, kn = ear.ear_kmeans(k, ki, w.iters)
+        (qc, ql, qn), (kc, kl, kn) = ear.ear_kmeans_pair(q, qi, k, ki, w.iters,
+                                                         streams=args.kmeans_streams)
         rec(1)
         if gathered:
             qp, qo, _, _ = ear.ear_permute(ql, w.c_q)
@@ -383,7 +384,7 @@ def run_ear(args, w):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded Gaussian-mixture / smoothed-field tokens; no model weights)",
-        "config": config_of(w, world, args.layout),
+        "config": config_of(w, world, args.layout, args.kmeans_streams),
         "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
         "overhead_frac": (stage_ms["kmeans"] + stage_ms["probe"] + stage_ms["route"]) /
                          sum(stage_ms.values()),
@@ -744,6 +745,8 @@ def main(argv=None):
                     help="run a quality study instead of the timing line")
     ap.add_argument("--c-q", type=int, default=None, help="query clusters of a study")
     ap.add_argument("--c-k", type=int, default=None, help="key clusters of a study")
+    ap.add_argument("--kmeans-streams", type=int, choices=(1, 2), default=2,
+                    help="Q's and K's k-means one after the other (1) or side by side (2)")
     ap.add_argument("--layout", choices=("permuted", "gathered"), default="permuted",
                     help="permuted copies of Q, K, V, or reads through the permutations")
     args = ap.parse_args(argv)

@@ -66,6 +66,36 @@ def ear_kmeans(x: torch.Tensor, init: torch.Tensor, iters: int):
     return cent, labels, counts
 
 
+_SIDE_STREAMS = {}
+
+
+def _side_stream(device) -> torch.cuda.Stream:
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _SIDE_STREAMS:
+        _SIDE_STREAMS[key] = torch.cuda.Stream(device=dev)
+    return _SIDE_STREAMS[key]
+
+
+def ear_kmeans_pair(q, q_init, k, k_init, iters: int, streams: int = 2):
+    """Q's and K's k-means (independent of each other, SVG-EAR §4.1).  With
+    streams=2, K's runs on a side stream beside Q's on the current stream and
+    the current stream waits for it before returning: each call's kernels fill
+    the other's tails and small launches.  Returns ((qc, ql, qn), (kc, kl, kn))."""
+    if streams == 1:
+        return ear_kmeans(q, q_init, iters), ear_kmeans(k, k_init, iters)
+    cur = torch.cuda.current_stream(q.device)
+    side = _side_stream(q.device)
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        kres = ear_kmeans(k, k_init, iters)
+    qres = ear_kmeans(q, q_init, iters)
+    cur.wait_stream(side)
+    for t in kres:
+        t.record_stream(cur)  # allocated on the side stream, used on this one
+    return qres, kres
+
+
 def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor] = None,
                 seg_mean: bool = False):
     """Stable cluster-contiguous permutation (SVG-EAR §3.1).
@@ -377,8 +407,7 @@ def ear_layer(q, k, v, q_init, k_init, iters: int, density: float, ratio_mode: i
     computed but never applied to a copy; the probe and the attention read rows
     through them (same results)."""
     n_q, n_k = q.shape[1], k.shape[1]
-    qc, ql, qn = ear_kmeans(q, q_init, iters)
-    kc, kl, kn = ear_kmeans(k, k_init, iters)
+    (qc, ql, qn), (kc, kl, kn) = ear_kmeans_pair(q, q_init, k, k_init, iters)
     if gather:
         qp, qo, _, _ = ear_permute(ql, q_init.shape[1])
         kp, ko, _, _ = ear_permute(kl, k_init.shape[1])
