@@ -77,23 +77,29 @@ def _side_stream(device) -> torch.cuda.Stream:
     return _SIDE_STREAMS[key]
 
 
-def ear_kmeans_pair(q, q_init, k, k_init, iters: int, streams: int = 2):
+def ear_kmeans_pair(q, q_init, k, k_init, iters: int, streams: int = 2, q_after=None):
     """Q's and K's k-means (independent of each other, SVG-EAR §4.1).  With
     streams=2, K's runs on a side stream beside Q's on the current stream and
     the current stream waits for it before returning: each call's kernels fill
-    the other's tails and small launches.  Returns ((qc, ql, qn), (kc, kl, kn))."""
+    the other's tails and small launches.  q_after(qc, ql, qn), if given, runs
+    on the current stream right after Q's k-means (under K's, which takes
+    longer); its result is returned third.
+    Returns ((qc, ql, qn), (kc, kl, kn), q_after's result or None)."""
     if streams == 1:
-        return ear_kmeans(q, q_init, iters), ear_kmeans(k, k_init, iters)
+        qres = ear_kmeans(q, q_init, iters)
+        kres = ear_kmeans(k, k_init, iters)
+        return qres, kres, (q_after(*qres) if q_after is not None else None)
     cur = torch.cuda.current_stream(q.device)
     side = _side_stream(q.device)
     side.wait_stream(cur)
     with torch.cuda.stream(side):
         kres = ear_kmeans(k, k_init, iters)
     qres = ear_kmeans(q, q_init, iters)
+    extra = q_after(*qres) if q_after is not None else None
     cur.wait_stream(side)
     for t in kres:
         t.record_stream(cur)  # allocated on the side stream, used on this one
-    return qres, kres
+    return qres, kres, extra
 
 
 def ear_permute(labels: torch.Tensor, n_clusters: int, x: Optional[torch.Tensor] = None,
@@ -407,14 +413,15 @@ def ear_layer(q, k, v, q_init, k_init, iters: int, density: float, ratio_mode: i
     computed but never applied to a copy; the probe and the attention read rows
     through them (same results)."""
     n_q, n_k = q.shape[1], k.shape[1]
-    (qc, ql, qn), (kc, kl, kn) = ear_kmeans_pair(q, q_init, k, k_init, iters)
+    # Q's permutation runs under K's k-means
+    q_perm = (lambda qc_, ql_, qn_: ear_permute(ql_, q_init.shape[1], None if gather else q))
+    (qc, ql, qn), (kc, kl, kn), (qp, qo, qx, _) = ear_kmeans_pair(q, q_init, k, k_init, iters,
+                                                                  q_after=q_perm)
     if gather:
-        qp, qo, _, _ = ear_permute(ql, q_init.shape[1])
         kp, ko, _, _ = ear_permute(kl, k_init.shape[1])
         _, vm = ear_permute_apply(kp, ko, v, seg_mean=True, write_perm=False)
         e = ear_probe_gather(qc, qn, kc, k, kp, ko, scale)
     else:
-        qp, qo, qx, _ = ear_permute(ql, q_init.shape[1], q)
         kp, ko, kx, _ = ear_permute(kl, k_init.shape[1], k)
         vx, vm = ear_permute_apply(kp, ko, v, seg_mean=True)
         e = ear_probe(qc, qn, kc, kx, ko, scale)
