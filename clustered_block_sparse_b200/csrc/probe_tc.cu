@@ -458,15 +458,18 @@ __global__ void pr_split(const float* __restrict__ qc, uint16_t* __restrict__ ou
 // -s μ_ab = -s q̄_a·k̄_b in fp64, stored as hi = fp32(value), lo = fp32(value - hi).
 // Block = (16 key clusters, a tile of 128 centroid rows, slice); thread = row a.
 // Layout [BH][C_k][mtiles * 128] (a fastest), so an epilogue warp reads it
-// coalesced.
+// coalesced.  k̄ is held in shared memory already widened to fp64 (one
+// conversion per value and block, not per value and thread); q̄'s rows are
+// padded to kM + 1 floats so its transposing stores do not share banks.
 constexpr int kMuB = 16;
+constexpr int kMuQS = kM + 1;
 template <int D>
 __global__ void __launch_bounds__(kM)
 pr_mu(const float* __restrict__ qc, const float* __restrict__ kc, int Cq, int Ck, int mtiles,
       double scale, float2* __restrict__ nmu) {
-  extern __shared__ float mu_smem[];
-  float (*qs)[kM] = reinterpret_cast<float (*)[kM]>(mu_smem);          // [D][kM]
-  float (*ks)[D] = reinterpret_cast<float (*)[D]>(mu_smem + D * kM);   // [kMuB][D]
+  extern __shared__ double mu_smem[];
+  double (*ks)[D] = reinterpret_cast<double (*)[D]>(mu_smem);                    // [kMuB][D]
+  float (*qs)[kMuQS] = reinterpret_cast<float (*)[kMuQS]>(mu_smem + kMuB * D);  // [D][kM + 1]
   const int b0 = blockIdx.x * kMuB;
   const int mt = blockIdx.y;
   const int64_t h = blockIdx.z;
@@ -477,7 +480,7 @@ pr_mu(const float* __restrict__ qc, const float* __restrict__ kc, int Cq, int Ck
   }
   for (int e = threadIdx.x; e < kMuB * D; e += kM) {
     const int bb = b0 + e / D;
-    ks[e / D][e % D] = bb < Ck ? kc[(h * Ck + bb) * (int64_t)D + e % D] : 0.f;
+    ks[e / D][e % D] = bb < Ck ? (double)kc[(h * Ck + bb) * (int64_t)D + e % D] : 0.0;
   }
   __syncthreads();
   double acc[kMuB];
@@ -486,7 +489,7 @@ pr_mu(const float* __restrict__ qc, const float* __restrict__ kc, int Cq, int Ck
   for (int k = 0; k < D; ++k) {
     const double qv = (double)qs[k][r];
 #pragma unroll
-    for (int i = 0; i < kMuB; ++i) acc[i] = fma(qv, (double)ks[i][k], acc[i]);
+    for (int i = 0; i < kMuB; ++i) acc[i] = fma(qv, ks[i][k], acc[i]);
   }
   const int apad = mtiles * kM;
 #pragma unroll
@@ -629,7 +632,7 @@ ear_status run_tc(const float* qc, const int32_t* qn, const float* kc, const voi
   const int64_t total = bh * mt * kParts * kM * D;
   pr_split<<<(unsigned)ceil_div(total, 256), 256, 0, s>>>(qc, w.qsplit, c_q, mt, D, total);
   EAR_TRY(after_launch());
-  const int mu_smem = (D * kM + kMuB * D) * (int)sizeof(float);
+  const int mu_smem = kMuB * D * (int)sizeof(double) + D * kMuQS * (int)sizeof(float);
   EAR_CUDA(cudaFuncSetAttribute(pr_mu<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, mu_smem));
   pr_mu<D><<<dim3((unsigned)ceil_div(c_k, kMuB), (unsigned)mt, (unsigned)bh), kM, mu_smem, s>>>(
       qc, kc, c_q, c_k, mt, (double)scale, w.nmu);
