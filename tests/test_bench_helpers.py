@@ -43,3 +43,36 @@ def test_config_names_the_workload():
     assert "no collective" in cfg["parallelism"]
     with pytest.raises(KeyError):
         bench.WORKLOADS["unknown"]
+
+
+def test_stage_bytes_count_each_copy_once():
+    """Q's permutation is timed in the k-means stage (it runs under K's
+    k-means), so its bytes are counted there: the layer total stays Q, K read
+    per k-means iteration, Q, K, V read and written once by the permutations,
+    K read by the probe, Q, K, V read and O written by the attention.  The
+    gathered layout writes no copy: 5 fewer passes over a token matrix (Q and
+    K read and written, V written) and V's permutation row bytes."""
+    bench = _load_bench(os.path.join(ROOT, "bench.py"))
+    w = bench.WORKLOADS["wan"]
+    tok = w.heads * w.n * w.d * 2
+    rows = w.heads * w.n
+    blocks = w.heads * w.c_q * w.c_k
+    p = bench.stage_bytes(w, "permuted")
+    g = bench.stage_bytes(w, "gathered")
+    kmeans = 2 * w.iters * (tok + 4 * rows)
+    permute = 6 * tok + 24 * rows
+    total = kmeans + permute + (tok + 4 * blocks) + 9 * blocks + 4 * tok
+    assert sum(p.values()) == total
+    assert p["kmeans"] == kmeans + 2 * tok + 8 * rows  # with Q's permutation
+    assert p["permute"] == 4 * tok + 16 * rows          # K's and V's
+    assert sum(p.values()) - sum(g.values()) == 5 * tok + 4 * rows
+    assert g["attention"] == p["attention"] == 4 * tok
+
+
+def test_config_records_the_layout_and_the_kmeans_schedule():
+    bench = _load_bench(os.path.join(ROOT, "bench.py"))
+    w = bench.WORKLOADS["wan"]
+    cfg = bench.config_of(w, 1, "gathered", 1)
+    assert cfg["layout"].startswith("gathered") and cfg["kmeans_streams"] == 1
+    cfg = bench.config_of(w, 1)
+    assert cfg["layout"].startswith("permuted") and cfg["kmeans_streams"] == 2
